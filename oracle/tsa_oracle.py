@@ -1,0 +1,216 @@
+"""Plain, slow, fp64 CPU oracle for the prefill attention of Token Sparse Attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import or call it.  It shares no code, table or
+helper with the CUDA library under ``long_context_tsa_b200/``; it never
+imports that package, and that package never imports this one.
+
+What it computes (each function cites the passage it follows):
+
+* ``score``   -- per-key importance: softmax of the scaled query-key logits
+  over the keys, summed over the queries.  Source: "Token Sparse Attention
+  Long Context" (skillsdirectory skill page), Step 1, ``TokenScorer.score_tokens``
+  with method "entropy".  Readings the page leaves open (stated in the
+  design notes): only the last ``window`` queries score (an observation
+  window), window query at position p sees keys j <= p (causal), and under
+  grouped-query attention the scores of the query heads that share a KV head
+  are summed.
+* ``select``  -- top-K per KV head.  Source: same page, Step 1,
+  ``TokenScorer.select_top_k`` (``torch.topk``) and Step 3 (K clamped to the
+  sequence length).  Reading: ties go to the lower index; the kept indices
+  are listed ascending, followed by the dropped indices ascending.
+* ``attend``  -- gather the kept rows of Q, K, V, run softmax attention on the
+  compressed tensors with a causal mask by original positions, and scatter the
+  result back to full length with zeros at dropped rows.  Source: same page,
+  Step 2 (``gather_tokens``, ``scatter_attention_output``) and Step 3
+  (``SparseAttentionHead.forward``); "Token Sparse Attention: Efficient
+  Long-Context Inference with Interleaved Token Selection" (sciencestack),
+  Figure 3 (compress Q/K/V per head, attend, scatter to the full sequence
+  layout before the residual add).
+
+All arithmetic is float64 on values widened exactly from the caller's inputs.
+Library primitives (``numpy.matmul``, ``numpy.argsort``) serve as single steps;
+there is no blocking or reordering beyond splitting rows into chunks to bound
+memory, which does not change any row's arithmetic.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+closed forms, invariants, brute force on tiny inputs and PyTorch's own
+scaled-dot-product attention.  The pages print no worked numeric example, so
+no end-to-end value is pinned by the pages themselves.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "clamp_budgets",
+    "score",
+    "select",
+    "attend",
+    "attend_rows",
+    "forward",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _scale(d: int, scale) -> float:
+    # Step 1 and Step 3 of the skill page divide the logits by the square root
+    # of the per-head dimension.
+    if scale is None or scale == 0.0:
+        return 1.0 / math.sqrt(d)
+    return float(scale)
+
+
+def clamp_budgets(budgets, L: int) -> np.ndarray:
+    """Kept-token count per (batch, KV head): ``min(budget, L)``.
+
+    The skill page's Step 3 passes ``k=min(self.k, seq_len)`` to the top-K.
+    A budget below 1 has no meaning on the pages and is rejected.
+    """
+    b = np.asarray(budgets, dtype=np.int64).reshape(-1)
+    if np.any(b < 1):
+        raise ValueError("every budget must be >= 1")
+    return np.minimum(b, L)
+
+
+def score(q, k, window: int, scale=None) -> np.ndarray:
+    """Per-KV-head token importance, shape [B, Hkv, L], float64.
+
+    For query head h (KV group g = h // G, G = Hq // Hkv) and each window query
+    at position p in [L - window, L):
+        logits_j = scale * q[p] . k[j]           for keys j <= p
+        prob_j   = softmax over those keys
+    and score_g[j] accumulates prob_j over the window queries of every query
+    head in group g.  Follows Step 1 ("entropy": matmul, divide by sqrt(d),
+    softmax over keys, sum over queries) with the window / causal / grouping
+    readings listed in the module docstring.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if not 1 <= window <= L:
+        raise ValueError("window must be in [1, L]")
+    G = Hq // Hkv
+    s = _scale(D, scale)
+    pos_q = np.arange(L - window, L)
+    visible = np.arange(L)[None, :] <= pos_q[:, None]  # [window, L]
+    out = np.zeros((B, Hkv, L), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            logits = s * (q[b, h, L - window:, :] @ k[b, g].T)  # [window, L]
+            logits = np.where(visible, logits, -np.inf)
+            m = logits.max(axis=1, keepdims=True)
+            e = np.exp(logits - m)
+            p = e / e.sum(axis=1, keepdims=True)
+            out[b, g] += p.sum(axis=0)
+    return out
+
+
+def select(scores, budgets) -> np.ndarray:
+    """Per-KV-head permutation of [0, L): kept indices ascending, then dropped ascending.
+
+    ``scores`` is [B, Hkv, L]; values are compared exactly in the dtype given
+    (pass float32 scores to reproduce a float32 decision).  The K = min(budget, L)
+    largest are kept; among equal values the lower index wins (a stable sort
+    on descending value).  Follows ``select_top_k`` (Step 1) with the tie and
+    ordering reading stated in the module docstring.  +0.0 and -0.0 compare
+    equal, as they do in IEEE arithmetic.
+    """
+    s = np.asarray(scores)
+    if s.ndim != 3:
+        raise ValueError("scores must be [B, Hkv, L]")
+    if not np.all(np.isfinite(s)):
+        raise ValueError("scores must be finite")
+    B, Hkv, L = s.shape
+    kept = clamp_budgets(budgets, L)
+    if kept.size != B * Hkv:
+        raise ValueError("one budget per (batch, KV head)")
+    perm = np.empty((B, Hkv, L), dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            K = int(kept[b * Hkv + g])
+            order = np.argsort(-s[b, g], kind="stable")
+            perm[b, g, :K] = np.sort(order[:K])
+            perm[b, g, K:] = np.sort(order[K:])
+    return perm
+
+
+def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=None) -> np.ndarray:
+    """Output rows for query head h of batch b at compacted indices ``rows``.
+
+    Compacted row i stands for original position p_i = perm_bg[i] (i < K).
+    Its output is  sum_r softmax_r(scale * q[p_i] . k[p_r]) * v[p_r]  over the
+    kept rows r whose original position p_r <= p_i (causal by original
+    positions).  Returns [len(rows), D] float64.  This is Step 3's
+    matmul / softmax / matmul on the gathered tensors of Step 2.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    D = q.shape[-1]
+    s = _scale(D, scale)
+    g = h // G
+    idx = np.asarray(perm_bg[:K], dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    kh = k[b, g, idx]  # [K, D]  gathered keys
+    vh = v[b, g, idx]  # [K, D]  gathered values
+    out = np.empty((rows.size, D), dtype=np.float64)
+    chunk = max(1, (1 << 22) // max(1, K))
+    for c0 in range(0, rows.size, chunk):
+        rr = rows[c0:c0 + chunk]
+        pq = idx[rr]  # original positions of these queries
+        qh = q[b, h, pq]  # [n, D]  gathered queries
+        logits = s * (qh @ kh.T)  # [n, K]
+        logits = np.where(idx[None, :] <= pq[:, None], logits, -np.inf)
+        m = logits.max(axis=1, keepdims=True)
+        e = np.exp(logits - m)
+        p = e / e.sum(axis=1, keepdims=True)
+        out[c0:c0 + chunk] = p @ vh
+    return out
+
+
+def attend(q, k, v, perm, budgets, scale=None) -> np.ndarray:
+    """Full output [B, Hq, L, D] float64: attention on the kept rows, zeros elsewhere.
+
+    Query head h uses the permutation and budget of its KV group h // G.
+    The attention output of kept row i is scattered to original position
+    perm[b, g, i]; every dropped position holds 0 (Step 2's
+    ``scatter_attention_output`` starts from a zero tensor).
+    """
+    q = _f64(q)
+    B, Hq, L, D = q.shape
+    Hkv = np.asarray(k).shape[1]
+    G = Hq // Hkv
+    kept = clamp_budgets(budgets, L)
+    perm = np.asarray(perm, dtype=np.int64)
+    out = np.zeros((B, Hq, L, D), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            K = int(kept[b * Hkv + g])
+            rows = np.arange(K)
+            out[b, h, perm[b, g, :K]] = attend_rows(q, k, v, perm[b, g], K, b, h, G, rows, scale)
+    return out
+
+
+def forward(q, k, v, window: int, budgets, scale=None):
+    """Score -> select (on float32-rounded scores) -> attend.  Returns (scores64, perm, out).
+
+    The selection runs on the scores rounded to float32, the precision in
+    which the library stores and compares them.
+    """
+    sc = score(q, k, window, scale)
+    perm = select(sc.astype(np.float32), budgets)
+    out = attend(q, k, v, perm, budgets, scale)
+    return sc, perm, out

@@ -1,0 +1,275 @@
+"""Pins for the fp64 oracle: each check is fixed by the pages or by mathematics,
+never by the oracle itself.
+
+Sources: "Token Sparse Attention Long Context" (skillsdirectory skill page),
+Step 1 (``score_tokens`` "entropy", ``select_top_k``), Step 2 (``gather_tokens``,
+``scatter_attention_output``), Step 3 (``SparseAttentionHead.forward``);
+"Token Sparse Attention: Efficient Long-Context Inference with Interleaved
+Token Selection" (sciencestack), Figure 3.
+
+The pages print no worked numeric example; the fixed values below are closed
+forms derived by hand, exhaustive enumeration on tiny inputs, and PyTorch's own
+scaled-dot-product attention (an independent library routine).
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tsa_oracle as O
+
+rng = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------------------- score
+
+
+def test_score_total_mass_is_window_times_group():
+    # Every window query's softmax sums to 1, so a KV group's scores sum to W * G.
+    B, Hq, Hkv, L, D, W = 2, 4, 2, 40, 8, 5
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    s = O.score(q, k, W)
+    assert s.shape == (B, Hkv, L)
+    np.testing.assert_allclose(s.sum(-1), W * (Hq // Hkv), rtol=0, atol=1e-12)
+    assert np.all(s >= 0)
+
+
+@pytest.mark.parametrize("W", [1, 3, 17, 24])
+def test_score_zero_queries_harmonic_closed_form(W):
+    # q = 0 makes every visible logit 0: the window query at position p spreads
+    # 1/(p+1) over keys 0..p.  So score_g[j] = G * sum_{p >= max(j, L-W)} 1/(p+1).
+    # Dropping the causal mask would give the flat value W*G/L instead.
+    B, Hq, Hkv, L, D = 1, 2, 1, 24, 4
+    q = np.zeros((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    s = O.score(q, k, W)
+    G = Hq // Hkv
+    want = np.array([G * sum(1.0 / (p + 1) for p in range(max(j, L - W), L)) for j in range(L)])
+    np.testing.assert_allclose(s[0, 0], want, rtol=1e-13, atol=1e-15)
+
+
+def test_score_two_token_hand_worked():
+    # L=2, W=2, d=4, scale 1/sqrt(4) = 1/2.  Query 0 sees only key 0 (prob 1).
+    # Query 1 = (2,0,0,0) against k0 = (1,0,0,0), k1 = 0: logits (1, 0), so
+    # prob(k0) = sigmoid(1).  score = (1 + sigmoid(1), 1 - sigmoid(1)).
+    q = np.zeros((1, 1, 2, 4))
+    q[0, 0, 0] = [0.3, -1.0, 2.0, 0.5]
+    q[0, 0, 1] = [2.0, 0.0, 0.0, 0.0]
+    k = np.zeros((1, 1, 2, 4))
+    k[0, 0, 0] = [1.0, 0.0, 0.0, 0.0]
+    sig1 = 0.7310585786300049  # 1 / (1 + e^-1)
+    s = O.score(q, k, 2)
+    np.testing.assert_allclose(s[0, 0], [1.0 + sig1, 1.0 - sig1], rtol=1e-14)
+    # An explicit scale of 1 doubles the logit: prob(k0) = sigmoid(2).
+    sig2 = 0.8807970779778823
+    s = O.score(q, k, 2, scale=1.0)
+    np.testing.assert_allclose(s[0, 0], [1.0 + sig2, 1.0 - sig2], rtol=1e-14)
+
+
+def test_score_gqa_groups_sum_their_own_query_heads():
+    # Hq=4, Hkv=2 (G=2): query heads 0,1 use KV head 0 and heads 2,3 use KV head 1.
+    # Keys are one-hot e_j; the last query of head h is a * e_{t_h}.  With W=1
+    # the only window query sees all 8 keys, logits a*s at t_h and 0 elsewhere:
+    # prob = e^{as}/(e^{as}+7) at t_h and 1/(e^{as}+7) elsewhere.
+    L, D, a = 8, 8, 5.0
+    t = [1, 2, 5, 6]
+    q = np.zeros((1, 4, L, D))
+    for h in range(4):
+        q[0, h, L - 1, t[h]] = a
+    k = np.zeros((1, 2, L, D))
+    k[0, :, np.arange(L), np.arange(L)] = 1.0
+    s = O.score(q, k, 1)
+    e = math.exp(a / math.sqrt(D))
+    hi, lo = e / (e + 7.0), 1.0 / (e + 7.0)
+    for g in range(2):
+        want = np.full(L, 2 * lo)
+        for h in (2 * g, 2 * g + 1):
+            want[t[h]] += hi - lo
+        np.testing.assert_allclose(s[0, g], want, rtol=1e-14)
+
+
+def test_score_only_window_queries_matter():
+    B, Hq, Hkv, L, D, W = 1, 2, 2, 30, 6, 7
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    s0 = O.score(q, k, W)
+    q2 = q.copy()
+    q2[:, :, : L - W] = rng.standard_normal((B, Hq, L - W, D))
+    np.testing.assert_array_equal(O.score(q2, k, W), s0)
+    q3 = q.copy()
+    q3[:, :, L - 1] += 1.0
+    assert not np.allclose(O.score(q3, k, W), s0)
+
+
+# ----------------------------------------------------------------------------- select
+
+
+def _brute_force_topk(vals, K):
+    # The max-sum K-subset; among equal sums the lexicographically smallest
+    # sorted index tuple (= ties broken toward lower indices).
+    best = None
+    for c in itertools.combinations(range(len(vals)), K):
+        key = (-sum(vals[i] for i in c), c)
+        if best is None or key < best:
+            best = key
+    return list(best[1])
+
+
+@pytest.mark.parametrize("L", range(1, 10))
+def test_select_matches_exhaustive_enumeration(L):
+    for trial in range(4):
+        vals = rng.integers(0, 4, size=L).astype(np.float64)  # many ties
+        for K in range(1, L + 1):
+            perm = O.select(vals[None, None, :], [K])[0, 0]
+            assert list(perm[:K]) == _brute_force_topk(list(vals), K)
+            assert sorted(perm.tolist()) == list(range(L))
+
+
+def test_select_invariants_random_and_ragged():
+    B, Hkv, L = 2, 3, 1000
+    s = rng.integers(0, 50, size=(B, Hkv, L)).astype(np.float32)
+    budgets = [1, 10, 999, 1000, 5000, 333]
+    perm = O.select(s, budgets)
+    for i, (b, g) in enumerate(itertools.product(range(B), range(Hkv))):
+        K = min(budgets[i], L)
+        p = perm[b, g]
+        assert sorted(p.tolist()) == list(range(L))
+        sel, rest = p[:K], p[K:]
+        assert np.all(np.diff(sel) > 0) and np.all(np.diff(rest) > 0)
+        if K < L:
+            thr = s[b, g, sel].min()
+            assert thr >= s[b, g, rest].max()
+            tied_sel = sel[s[b, g, sel] == thr]
+            tied_rest = rest[s[b, g, rest] == thr]
+            if tied_rest.size:
+                assert tied_sel.max() < tied_rest.min()
+
+
+def test_select_clamps_budget_to_length_and_rejects_nonpositive():
+    s = rng.random((1, 1, 12)).astype(np.float32)
+    np.testing.assert_array_equal(O.select(s, [99])[0, 0], np.arange(12))
+    with pytest.raises(ValueError):
+        O.select(s, [0])
+
+
+def test_select_signed_zero_ties_and_last_bit():
+    s = np.array([[[-0.0, 0.0, 1.0, -0.0, 0.0]]], dtype=np.float32)
+    assert O.select(s, [3])[0, 0, :3].tolist() == [0, 1, 2]
+    a = np.float32(0.1)
+    b = np.nextafter(a, np.float32(1.0))  # one ulp larger in float32
+    s = np.array([[[a, a, b, a]]], dtype=np.float32)
+    assert O.select(s, [1])[0, 0, :1].tolist() == [2]
+    assert O.select(s, [2])[0, 0, :2].tolist() == [0, 2]
+
+
+# ----------------------------------------------------------------------------- attend
+
+
+def _sdpa64(q, k, v, mask=None, causal=False, scale=None):
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))  # noqa: E731
+    G = q.shape[1] // k.shape[1]
+    out = torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=None if mask is None else torch.from_numpy(mask),
+        is_causal=causal, scale=scale, enable_gqa=G > 1)
+    return out.numpy()
+
+
+def test_attend_keep_all_is_dense_causal_attention():
+    # K = L: gather and scatter are identities and the op is ordinary causal
+    # attention (Step 3 on the full token set), checked against PyTorch SDPA,
+    # whose grouped-query mode maps query head h to KV head h // G.
+    B, Hq, Hkv, L, D = 2, 4, 2, 50, 16
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    perm = np.broadcast_to(np.arange(L), (B, Hkv, L))
+    out = O.attend(q, k, v, perm, [L] * (B * Hkv))
+    np.testing.assert_allclose(out, _sdpa64(q, k, v, causal=True), rtol=0, atol=1e-12)
+
+
+def test_attend_equals_full_length_masked_attention():
+    # Attention on the compressed tensors equals full-length attention with the
+    # mask M[p, r] = kept[r] and r <= p, read at the kept rows; dropped rows are 0.
+    B, Hq, Hkv, L, D = 1, 4, 2, 40, 8
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    budgets = [13, 29]
+    perm = O.select(rng.random((B, Hkv, L)), budgets)
+    out = O.attend(q, k, v, perm, budgets)
+    G = Hq // Hkv
+    for g in range(Hkv):
+        kept = np.zeros(L, bool)
+        kept[perm[0, g, : budgets[g]]] = True
+        mask = kept[None, :] & (np.arange(L)[None, :] <= np.arange(L)[:, None])
+        hs = slice(g * G, (g + 1) * G)
+        ref = _sdpa64(q[:, hs], k[:, g:g + 1], v[:, g:g + 1], mask=mask)
+        np.testing.assert_allclose(out[0, hs][:, kept], ref[0][:, kept], rtol=0, atol=1e-12)
+        assert np.all(out[0, hs][:, ~kept] == 0.0)
+
+
+def test_attend_first_kept_row_copies_its_value_row():
+    B, Hq, Hkv, L, D = 1, 2, 1, 20, 4
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    perm = O.select(rng.random((B, Hkv, L)), [7])
+    out = O.attend(q, k, v, perm, [7])
+    p0 = perm[0, 0, 0]
+    for h in range(Hq):
+        np.testing.assert_array_equal(out[0, h, p0], v[0, 0, p0])
+
+
+def test_attend_zero_queries_give_prefix_means():
+    B, Hq, Hkv, L, D, K = 1, 1, 1, 30, 5, 11
+    q = np.zeros((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    perm = O.select(rng.random((B, Hkv, L)), [K])
+    out = O.attend(q, k, v, perm, [K])
+    vh = v[0, 0, perm[0, 0, :K]]
+    want = np.cumsum(vh, axis=0) / np.arange(1, K + 1)[:, None]
+    np.testing.assert_allclose(out[0, 0, perm[0, 0, :K]], want, rtol=1e-13, atol=1e-14)
+
+
+def test_attend_rows_within_convex_hull_and_subset_agrees():
+    B, Hq, Hkv, L, D, K = 1, 2, 1, 64, 8, 33
+    q = 3.0 * rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    perm = O.select(rng.random((B, Hkv, L)), [K])
+    out = O.attend(q, k, v, perm, [K])
+    vh = v[0, 0, perm[0, 0, :K]]
+    for i in range(K):
+        row = out[0, 1, perm[0, 0, i]]
+        assert np.all(row <= vh[: i + 1].max(0) + 1e-12)
+        assert np.all(row >= vh[: i + 1].min(0) - 1e-12)
+    rows = np.array([0, 5, 32])
+    sub = O.attend_rows(q, k, v, perm[0, 0], K, 0, 1, 2, rows)
+    np.testing.assert_allclose(sub, out[0, 1, perm[0, 0, rows]], rtol=0, atol=1e-14)
+
+
+def test_forward_preserves_shape_and_composes():
+    B, Hq, Hkv, L, D, W = 1, 4, 2, 48, 8, 6
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    sc, perm, out = O.forward(q, k, v, W, [12, 20])
+    assert out.shape == (B, Hq, L, D)
+    np.testing.assert_array_equal(perm, O.select(O.score(q, k, W).astype(np.float32), [12, 20]))
+    np.testing.assert_array_equal(out, O.attend(q, k, v, perm, [12, 20]))
+
+
+def test_attend_budget_above_length_is_clamped():
+    # Step 3 of the skill page clamps the kept count to the sequence length.
+    B, Hq, Hkv, L, D = 1, 2, 1, 16, 4
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    perm = np.broadcast_to(np.arange(L), (B, Hkv, L))
+    np.testing.assert_array_equal(O.attend(q, k, v, perm, [10 * L]), O.attend(q, k, v, perm, [L]))
+    assert O.clamp_budgets([10 * L, 3], L).tolist() == [L, 3]
