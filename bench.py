@@ -1,0 +1,434 @@
+"""Benchmark of the Token Sparse Attention prefill hot path on B200.
+
+One step = the whole hot path over one layer of the L=131072 workload
+(B=1, 32 query / 8 KV heads, d=128, bf16, window 64, keep 0.1 per KV head):
+tsa_score -> tsa_select -> tsa_attend (gather, causal attention on the
+compressed tensors, scatter + zero fill), with inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tsa|reference]
+
+N > 1 runs under torchrun, one independent layer per rank (weak scaling, no
+collective on the data path); the step time is the max over ranks of the
+device-timed region.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference the pages
+allow: their authors' kernels are not available) on a bounded sample of the
+same workload, scaled to the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-attention prefill tokens/s at 128K; TFLOPS and % of B200 bf16 peak"
+WORKLOAD = "gqa_bf16_L131072"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+
+def attend_flops(w, budgets) -> float:
+    """Compacted causal attention flops: per query head, QK^T and PV over the
+    lower triangle including the diagonal, 2 flops per multiply-add."""
+    total = 0.0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            K = min(budgets[b * w.Hkv + g], w.L)
+            total += w.G * 4.0 * w.D * K * (K + 1) / 2.0
+    return total
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel_tag: str, workload: str, src_files):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (its sha256 is recorded in the summary)."""
+    digest = hashlib.sha256()
+    for f in src_files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            digest.update(fh.read())
+    want = digest.hexdigest()[:16]
+    for path in glob.glob(os.path.join(ROOT, "profiles", f"{kernel_tag}*{workload}*.md")):
+        text = open(path).read()
+        m_src = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+        m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        if m_src and m_tr and m_src.group(1) == want:
+            return float(m_tr.group(1)), os.path.relpath(path, ROOT)
+    return None, None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        props = torch.cuda.get_device_properties(self.device)
+        bus = getattr(props, "pci_bus_id", None)
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    pci_bus = int(parts[0].split(":")[1], 16)
+                except Exception:
+                    pci_bus = None
+                if bus is not None and pci_bus is not None and pci_bus != bus:
+                    continue
+                rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        # Samples are at 50 ms; drop the idle ones before/after the load.
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+
+def oracle_sample(w, q, k, v, budgets, heads, rows_per_head, seed=0):
+    """Time the oracle on a bounded sample and scale it to one full step.
+
+    score: `heads` query heads of the window (scaled to all Hq heads);
+    select: the KV groups of those heads (scaled to all B*Hkv groups);
+    attend: `rows_per_head` kept rows of each sampled head (scaled to all kept rows).
+    q, k, v: host float32 arrays.
+    """
+    from oracle import tsa_oracle as O
+
+    rng = np.random.default_rng(seed)
+    hs = sorted(rng.choice(w.Hq, size=min(heads, w.Hq), replace=False).tolist())
+    groups = sorted({h // w.G for h in hs})
+    t0 = time.perf_counter()
+    sc = {}
+    for h in hs:
+        g = h // w.G
+        part = O.score(q[:, h:h + 1], k[:, g:g + 1], w.W)
+        sc[g] = sc.get(g, 0.0) + part[0, 0]
+    t1 = time.perf_counter()
+    perms = {}
+    for g in groups:
+        perms[g] = O.select(np.asarray(sc[g], dtype=np.float32)[None, None, :], [budgets[g]])[0, 0]
+    t2 = time.perf_counter()
+    n_rows = 0
+    for h in hs:
+        g = h // w.G
+        K = min(budgets[g], w.L)
+        rows = rng.choice(K, size=min(rows_per_head, K), replace=False)
+        O.attend_rows(q, k, v, perms[g], K, 0, h, w.G, rows)
+        n_rows += rows.size
+    t3 = time.perf_counter()
+    total_rows = sum(w.G * min(budgets[g], w.L) for g in range(w.B * w.Hkv))
+    est = (t1 - t0) * (w.B * w.Hq / len(hs)) + (t2 - t1) * (w.B * w.Hkv / len(groups)) + \
+        (t3 - t2) * (total_rows / max(1, n_rows))
+    sample = (f"score {len(hs)}/{w.B * w.Hq} query heads (x{w.B * w.Hq / len(hs):.0f}), select "
+              f"{len(groups)}/{w.B * w.Hkv} KV groups (x{w.B * w.Hkv / len(groups):.0f}), attend {n_rows} of "
+              f"{total_rows} kept rows (x{total_rows / max(1, n_rows):.1f}); fp64 numpy")
+    return est, t3 - t0, sample
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tsa", choices=["tsa", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from long_context_tsa_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = I.WORKLOADS[args.workload]
+    budgets = w.budgets(seed=0)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args, w, budgets, world)
+        return
+
+    import long_context_tsa_b200 as T
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    q, k, v = I.make_qkv(w, seed=rank, device=dev)
+    desc = T.desc_for(q, k)
+    ws = T.alloc_workspace(desc, w.W, device=dev)
+    scores = torch.empty((w.B, w.Hkv, w.L), dtype=torch.float32, device=dev)
+    perm = torch.empty((w.B, w.Hkv, w.L), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        T.tsa_score(desc, q, k, w.W, scores, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        T.tsa_select(desc, scores, budgets, perm, ws)
+        if ev is not None:
+            ev[2].record(stream)
+        T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = T.tsa_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {T.tsa_status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = T.tsa_debug_launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = T.tsa_debug_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    st = T.tsa_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {T.tsa_status_string(st)}")
+
+    total_ms = start.elapsed_time(end)
+    t_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    t_attend = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    if dist is not None:
+        t = torch.tensor([total_ms, t_attend], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, t_attend = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    tokens = w.B * w.L
+    value = world * tokens / (ms_per_step / 1e3)
+
+    peaks, peak_src = load_peaks()
+    flops = attend_flops(w, budgets)
+    achieved = flops / (t_attend / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_simt.cu"])
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(T, w, desc, q, k, v, budgets, dev, stream, args.e2e_steps, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qn, kn, vn = (t.float().cpu().numpy() for t in (q, k, v))
+        est, wall, sample = oracle_sample(w, qn, kn, vn, budgets, heads=w.Hq, rows_per_head=256)
+        cpu = {"value": tokens / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": sample + f"; {wall:.1f} s of CPU work, estimated full step {est:.1f} s"}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+                   "K_per_kv_head": budgets, "l2": "inputs larger than L2 (q 1.07 GB, k and v 268 MB each)",
+                   "parallelism": f"{world} independent layers, one per GPU"},
+        "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend},
+        "attend_tflops": achieved,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": f"bf16_tflops ({peak_src})",
+                     "kernel": "tsa_attend", "traffic_source": traffic_src},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": launches,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist):
+    """Same metric through tsa_forward_host: pinned host inputs copied in, the
+    forward, and the full output copied back, all inside the timed region."""
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    qd, kd, vd, od = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(q)
+    ws = T.alloc_workspace(desc, w.W, device=dev)
+    for _ in range(2):
+        T.tsa_forward_host(desc, qh, kh, vh, w.W, budgets, oh, qd, kd, vd, od, ws)
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    s.record(stream)
+    for _ in range(steps):
+        T.tsa_forward_host(desc, qh, kh, vh, w.W, budgets, oh, qd, kd, vd, od, ws)
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    st = T.tsa_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after e2e: {T.tsa_status_string(st)}")
+    world = dist.get_world_size() if dist is not None else 1
+    nb = lambda t: t.numel() * t.element_size()  # noqa: E731
+    return {"value": world * w.B * w.L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
+            "d2h_bytes_per_step": nb(q), "ms_per_step": ms, "steps": steps}
+
+
+def run_reference(args, w, budgets, world):
+    """The oracle arm: W warm-up and K timed steps, each a bounded sample of the
+    workload scaled to one full step, on the host cores (rank 0 only)."""
+    from long_context_tsa_b200 import inputs as I
+
+    q, k, v = I.make_qkv(w, seed=0, device="cpu")
+    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
+    ests = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        est, wall, sample = oracle_sample(w, qn, kn, vn, budgets, heads=1, rows_per_head=256, seed=i)
+        if i >= args.warmup:
+            ests.append(est)
+    ms = statistics.mean(ests) * 1e3
+    value = w.B * w.L / (ms / 1e3)
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+                   "K_per_kv_head": budgets},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample + " per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * tsa.h -- C ABI of the Token Sparse Attention prefill hot path (sm_100a).
+ *
+ * The operation is the per-layer prefill attention of Token Sparse Attention:
+ * every KV head scores all L tokens, keeps its own top-K subset, compresses
+ * Q/K/V to that subset, runs causal attention on the compressed tensors and
+ * scatters the result back to length L (zeros at dropped rows), ready for the
+ * caller's residual add.
+ *
+ * Sources (page title, then the section / figure):
+ *   [P1] "Token Sparse Attention Long Context" (skillsdirectory skill page):
+ *        Step 1 TokenScorer.score_tokens ("entropy") and select_top_k;
+ *        Step 2 gather_tokens and scatter_attention_output;
+ *        Step 3 SparseAttentionHead.forward.
+ *   [P2] "Token Sparse Attention: Efficient Long-Context Inference with
+ *        Interleaved Token Selection" (sciencestack): Figure 3 (Stage 1
+ *        compresses Q, K, V per head to a token subset; Stage 2 attends on the
+ *        compressed tensors and scatters back to the full sequence layout
+ *        before the residual add); TL;DR (head-specific subsets).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Layout, row-major and contiguous ("BHLD"):
+ *     q   [B, Hq,  L, D]     k, v [B, Hkv, L, D]     out [B, Hq, L, D]
+ *     scores [B, Hkv, L] float32      perm [B, Hkv, L] int32
+ *   dtype of q/k/v/out: TSA_F32 (float) or TSA_BF16 (bfloat16).
+ *   Query head h belongs to KV group g = h / G, G = Hq / Hkv.
+ * - Every tensor pointer is DEVICE memory owned by the caller, 16-byte aligned.
+ *   The library allocates nothing, frees nothing and does not synchronise in
+ *   the compute calls: work is enqueued on `stream` (a cudaStream_t passed as
+ *   void*, NULL = legacy default stream) and the call returns.
+ * - `budget_host` is a HOST array of B*Hkv int32 kept-token counts, one per
+ *   (batch, KV head), read during the call (grid planning needs it).  A budget
+ *   <= 0 is TSA_ERR_INVALID_ARG; a budget > L is clamped to L, as [P1] Step 3
+ *   clamps k to the sequence length.
+ * - `ws` is a device workspace of at least tsa_workspace_size() bytes, owned by
+ *   the caller, zero-filled once before first use (tsa_workspace_init).  It
+ *   holds a device status word; calls sharing one workspace must be ordered on
+ *   one stream.
+ * - Argument errors are returned synchronously and nothing is launched.
+ *   Device-side errors (a bounded wait that ran out, a failed bounds check)
+ *   are recorded in the workspace status word and reported by
+ *   tsa_check_status().
+ * - Supported: D in {64, 128}; Hq % Hkv == 0; G = Hq/Hkv in {1,2,4,8,16};
+ *   1 <= window <= L; G*window <= 256; B*Hq*L < 2^31.
+ *   bf16 runs on tcgen05 tensor-core kernels, f32 on exact SIMT kernels.
+ *   There is no CPU path.
+ */
+#ifndef TSA_H_
+#define TSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TSA_API __attribute__((visibility("default")))
+#else
+#define TSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tsa_status {
+  TSA_OK = 0,
+  TSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or budget   */
+  TSA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes/dtypes */
+  TSA_ERR_WORKSPACE = 3,     /* workspace smaller than tsa_workspace_size()   */
+  TSA_ERR_CUDA = 4,          /* a CUDA runtime call failed                    */
+  TSA_ERR_TIMEOUT = 5,       /* a device-side bounded wait ran out            */
+  TSA_ERR_DEVICE_BOUNDS = 6  /* a device-side index check failed              */
+} tsa_status;
+
+typedef enum tsa_dtype { TSA_F32 = 0, TSA_BF16 = 1 } tsa_dtype;
+
+/* Problem shape.  scale <= 0 selects 1/sqrt(D), the 1/sqrt(head dim) of
+ * [P1] Step 1 and Step 3. */
+typedef struct tsa_desc {
+  int32_t B, Hq, Hkv, L, D;
+  int32_t dtype; /* tsa_dtype */
+  float scale;
+} tsa_desc;
+
+/* Bytes of device workspace needed by any call on this shape and window. */
+TSA_API size_t tsa_workspace_size(const tsa_desc* desc, int32_t window);
+
+/* Zero the workspace header (status word, counters).  Enqueued on `stream`. */
+TSA_API tsa_status tsa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_score -- per-KV-head token importance ([P1] Step 1, "entropy":
+ * softmax of q.k/sqrt(d) over keys, summed over queries).
+ * For each query head h and each of the last `window` query positions
+ * p in [L-window, L): logits_j = scale * q[p].k[j] over keys j <= p, softmax
+ * over j, accumulated into scores[b, h/G, j] (summed over the window queries
+ * and over the G query heads of the KV group).  Each KV head's scores sum to
+ * window*G.  Output: scores [B,Hkv,L] float32, fully overwritten.
+ */
+TSA_API tsa_status tsa_score(const tsa_desc* desc, const void* q, const void* k, int32_t window,
+                     float* scores, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_select -- top-K per KV head ([P1] Step 1 select_top_k; [P2] Figure 3
+ * per-head subsets; budgets may differ per head).  For (b,g) with
+ * K = min(budget_host[b*Hkv+g], L): keeps the K largest scores, ties broken
+ * toward the lower index, +0.0 == -0.0.  perm[b,g,0:K] lists the kept token
+ * indices ascending, perm[b,g,K:L] the dropped ones ascending.  Scores must
+ * be finite.  Bit-exact and deterministic.
+ */
+TSA_API tsa_status tsa_select(const tsa_desc* desc, const float* scores, const int32_t* budget_host,
+                      int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_attend -- gather, causal attention on the compressed tensors, scatter
+ * ([P1] Steps 2-3; [P2] Figure 3 Stages 1-2).  For query head h, group g,
+ * K = min(budget, L), kept row i < K at original position p_i = perm[b,g,i]:
+ *   out[b,h,p_i] = sum_{r <= i} softmax_r(scale * q[b,h,p_i].k[b,g,p_r]) v[b,g,p_r]
+ * (causal by original positions; perm[b,g,0:K] must be strictly ascending).
+ * Every dropped position perm[b,g,K:L] gets +0 in all D columns.  `out` is
+ * fully overwritten.  perm must be a permutation of [0,L) per (b,g) in the
+ * layout tsa_select produces; indices outside [0,L) are a device bounds error.
+ */
+TSA_API tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                      const int32_t* perm, const int32_t* budget_host, void* out, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * tsa_forward -- tsa_score, tsa_select and tsa_attend in sequence on `stream`.
+ * scores_or_null / perm_or_null: where to keep the intermediates; NULL puts
+ * them in the workspace.
+ */
+TSA_API tsa_status tsa_forward(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                       int32_t window, const int32_t* budget_host, float* scores_or_null,
+                       int32_t* perm_or_null, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_forward_host -- tsa_forward on HOST inputs and output.  q_host/k_host/
+ * v_host are copied into the caller's device buffers q_dev/k_dev/v_dev with
+ * one cudaMemcpyAsync each, the forward runs, and out_dev is copied back to
+ * out_host; all on `stream`.  The call returns after enqueueing; the host
+ * buffers must stay valid (and should be pinned for asynchrony) until the
+ * stream reaches that point.
+ */
+TSA_API tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void* k_host,
+                            const void* v_host, int32_t window, const int32_t* budget_host,
+                            void* out_host, void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, return the device status recorded in `ws` (TSA_OK,
+ * TSA_ERR_TIMEOUT or TSA_ERR_DEVICE_BOUNDS) and clear it. */
+TSA_API tsa_status tsa_check_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Static description of a status code. */
+TSA_API const char* tsa_status_string(tsa_status s);
+
+/*
+ * Failure-detection and accounting hooks (testing; no counterpart on the pages).
+ * tsa_debug_set_wait_limit: poll budget of every device-side bounded wait of
+ *   later launches in this process (0 restores the default of about a second).
+ * tsa_debug_wait_never_set: launch one block that waits on a workspace flag
+ *   nothing sets; with a small limit it records TSA_ERR_TIMEOUT and returns.
+ */
+TSA_API void tsa_debug_set_wait_limit(uint64_t polls);
+/* Number of kernels this library has launched in this process (all devices). */
+TSA_API uint64_t tsa_debug_launch_count(void);
+TSA_API tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSA_H_ */

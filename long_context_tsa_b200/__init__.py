@@ -1,0 +1,29 @@
+"""Token Sparse Attention prefill hot path on B200 (sm_100a).
+
+The compute lives in ``libtsa.so`` (CUDA kernels behind the C ABI of
+``include/tsa.h``); ``_native`` is its ctypes binding.  Importing this package
+does not load the library; the first call does, and fails loudly if it is
+missing.
+"""
+
+from ._native import (  # noqa: F401
+    TSA_BF16,
+    TSA_F32,
+    TsaDesc,
+    TsaError,
+    alloc_workspace,
+    desc_for,
+    make_desc,
+    tsa_attend,
+    tsa_check_status,
+    tsa_debug_launch_count,
+    tsa_debug_set_wait_limit,
+    tsa_debug_wait_never_set,
+    tsa_forward,
+    tsa_forward_host,
+    tsa_score,
+    tsa_select,
+    tsa_status_string,
+    tsa_workspace_init,
+    tsa_workspace_size,
+)

@@ -1,0 +1,172 @@
+"""ctypes binding of libtsa.so: the C entry points under the same names.
+
+Argument marshalling only -- every step runs in the CUDA kernels of the
+library.  Tensors are PyTorch tensors (device memory for the compute calls,
+host memory for ``tsa_forward_host``); budgets are Python sequences of ints.
+There is no fallback: a missing library raises ``RuntimeError``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtsa.so")
+
+TSA_F32, TSA_BF16 = 0, 1
+STATUS_NAMES = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_UNSUPPORTED", 3: "TSA_ERR_WORKSPACE",
+                4: "TSA_ERR_CUDA", 5: "TSA_ERR_TIMEOUT", 6: "TSA_ERR_DEVICE_BOUNDS"}
+STATUS = {v: k for k, v in STATUS_NAMES.items()}
+
+EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select", "tsa_attend", "tsa_forward",
+            "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
+            "tsa_debug_wait_never_set", "tsa_debug_launch_count")
+
+
+class TsaDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("L", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class TsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "tsa_workspace_size": (_SZ, [ctypes.POINTER(TsaDesc), _I32]),
+    "tsa_workspace_init": (ctypes.c_int, [_P, _SZ, _P]),
+    "tsa_score": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P, _SZ, _P]),
+    "tsa_select": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _SZ, _P]),
+    "tsa_attend": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tsa_forward": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tsa_forward_host": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _P,
+                                        _SZ, _P]),
+    "tsa_check_status": (ctypes.c_int, [_P, _SZ, _P]),
+    "tsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "tsa_debug_set_wait_limit": (None, [ctypes.c_uint64]),
+    "tsa_debug_wait_never_set": (ctypes.c_int, [_P, _SZ, _P]),
+    "tsa_debug_launch_count": (ctypes.c_uint64, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtsa.so (built in-tree by ``long_context_tsa_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA extension missing: {LIB_PATH} (run python -m long_context_tsa_b200.build)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _budgets(b):
+    arr = (ctypes.c_int32 * len(b))(*[int(x) for x in b])
+    return arr
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise TsaError(code, where)
+
+
+def make_desc(B: int, Hq: int, Hkv: int, L: int, D: int, dtype, scale: float = 0.0) -> TsaDesc:
+    if isinstance(dtype, torch.dtype):
+        dtype = TSA_F32 if dtype == torch.float32 else TSA_BF16 if dtype == torch.bfloat16 else -1
+    return TsaDesc(B, Hq, Hkv, L, D, int(dtype), float(scale))
+
+
+def desc_for(q: torch.Tensor, k: torch.Tensor, scale: float = 0.0) -> TsaDesc:
+    B, Hq, L, D = q.shape
+    return make_desc(B, Hq, k.shape[1], L, D, q.dtype, scale)
+
+
+def tsa_workspace_size(desc: TsaDesc, window: int) -> int:
+    return int(lib().tsa_workspace_size(ctypes.byref(desc), int(window)))
+
+
+def tsa_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().tsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "tsa_workspace_init")
+
+
+def alloc_workspace(desc: TsaDesc, window: int, device="cuda") -> torch.Tensor:
+    """Caller-side workspace allocation (PyTorch owns the memory), zero-filled."""
+    n = tsa_workspace_size(desc, window)
+    if n == 0:
+        raise TsaError(STATUS["TSA_ERR_INVALID_ARG"], "tsa_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def tsa_score(desc, q, k, window, scores, ws, stream=None):
+    _check(lib().tsa_score(ctypes.byref(desc), _ptr(q), _ptr(k), int(window), _ptr(scores), _ptr(ws),
+                           ws.numel(), _stream(stream)), "tsa_score")
+
+
+def tsa_select(desc, scores, budgets, perm, ws, stream=None):
+    _check(lib().tsa_select(ctypes.byref(desc), _ptr(scores), _budgets(budgets), _ptr(perm), _ptr(ws), ws.numel(),
+                            _stream(stream)), "tsa_select")
+
+
+def tsa_attend(desc, q, k, v, perm, budgets, out, ws, stream=None):
+    _check(lib().tsa_attend(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
+                            _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "tsa_attend")
+
+
+def tsa_forward(desc, q, k, v, window, budgets, out, ws, scores=None, perm=None, stream=None):
+    _check(lib().tsa_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), int(window), _budgets(budgets),
+                             _ptr(scores), _ptr(perm), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "tsa_forward")
+
+
+def tsa_forward_host(desc, q_host, k_host, v_host, window, budgets, out_host, q_dev, k_dev, v_dev, out_dev, ws,
+                     stream=None):
+    _check(lib().tsa_forward_host(ctypes.byref(desc), _ptr(q_host), _ptr(k_host), _ptr(v_host), int(window),
+                                  _budgets(budgets), _ptr(out_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                  _ptr(out_dev), _ptr(ws), ws.numel(), _stream(stream)), "tsa_forward_host")
+
+
+def tsa_check_status(ws, stream=None) -> int:
+    """Synchronise, return the device status code recorded in ``ws`` (0 = ok) and clear it."""
+    return int(lib().tsa_check_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def tsa_status_string(code: int) -> str:
+    return lib().tsa_status_string(int(code)).decode()
+
+
+def tsa_debug_set_wait_limit(polls: int):
+    lib().tsa_debug_set_wait_limit(int(polls))
+
+
+def tsa_debug_wait_never_set(ws, stream=None):
+    _check(lib().tsa_debug_wait_never_set(_ptr(ws), ws.numel(), _stream(stream)), "tsa_debug_wait_never_set")
+
+
+def tsa_debug_launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().tsa_debug_launch_count())

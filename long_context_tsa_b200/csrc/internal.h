@@ -1,0 +1,56 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/tsa.h"
+
+namespace tsa {
+
+constexpr int kMaxGroups = 1024;      // B * Hkv limit (budgets travel as kernel parameters)
+constexpr int kMaxWindowRows = 256;   // G * window limit
+constexpr int kScoreKeyTile = 64;     // keys per SIMT score tile
+constexpr int kMaxScoreSplits = 256;  // key-range splits per KV head in the score passes
+
+struct Dims {
+  int B, Hq, Hkv, L, D, G, dtype;
+  float scale;  // resolved (> 0)
+};
+
+// Workspace regions, byte offsets from the workspace base (256-byte aligned).
+struct WsLayout {
+  size_t status;  // uint32 status word + counters (256 B header)
+  size_t scores;  // [B,Hkv,L] f32 scratch for tsa_forward
+  size_t perm;    // [B,Hkv,L] i32 scratch for tsa_forward
+  size_t part;    // score partials [B*Hkv][splits][Mp] x {max, sum} f32
+  size_t lse;     // combined per-row log-normaliser [B*Hkv][Mp] f32
+  size_t total;
+};
+
+WsLayout ws_layout(const Dims& d, int window);
+int score_splits(const Dims& d);
+int window_rows_padded(const Dims& d, int window);  // Mp: G*window rounded up to 64
+
+uint64_t wait_limit();  // polls for device bounded waits
+void count_launches(int n);  // every launcher reports the kernels it enqueued
+
+// Kept counts clamped to L, one per (b, g); filled by the host entry points.
+struct Budgets {
+  int32_t kept[kMaxGroups];
+};
+
+// ---- launchers (return the CUDA error of the launch) ----
+cudaError_t launch_score_simt(const Dims& d, const void* q, const void* k, int window, float* scores,
+                              float* part, uint32_t* status, cudaStream_t st);
+cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kept, int32_t* perm,
+                          uint32_t* status, cudaStream_t st);
+cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
+                               const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
+                               cudaStream_t st);
+cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
+                             uint32_t* status, cudaStream_t st);
+cudaError_t launch_debug_wait(uint32_t* status, uint32_t* flag, uint64_t limit, cudaStream_t st);
+
+}  // namespace tsa

@@ -1,0 +1,220 @@
+// Top-K token selection per KV head: radix select + stable compaction.
+//
+// "Token Sparse Attention Long Context" (skill page), Step 1 select_top_k,
+// with per-head budgets ("Token Sparse Attention: Efficient Long-Context
+// Inference with Interleaved Token Selection", Figure 3: a token subset per
+// head).  For each (b, g) with K kept tokens the kernel finds the exact
+// 32-bit key T of the K-th largest score, keeps every score above T and the
+// first (in index order) of those equal to T, and writes
+//   perm[0:K]  = kept indices ascending,   perm[K:L] = dropped indices ascending.
+//
+// One thread-block cluster of kClusterCtas CTAs per (b, g); CTA `rank` owns a
+// contiguous index slice.  Four 8-bit radix passes build per-CTA shared-memory
+// histograms that every CTA sums over the cluster through distributed shared
+// memory; each CTA then derives the same digit.  Compaction: the kept position
+// of index i is  #(keys > T before i) + min(#(keys == T before i), ties_left),
+// a block-wide scan per chunk plus the slice offsets exchanged over the cluster.
+#include <cooperative_groups.h>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace tsa {
+namespace {
+
+constexpr int kClusterCtas = 8;
+constexpr int kThreads = 1024;
+constexpr int kPerThread = 4;
+constexpr int kChunk = kThreads * kPerThread;
+
+struct SelectArgs {
+  const float* scores;
+  int32_t* perm;
+  uint32_t* status;
+  int L, Hkv;
+  Budgets kept;
+};
+
+// Exclusive block scan of one u32 per thread (all kThreads threads call it).
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = warp_sums[lane];  // kThreads / 32 == 32 warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const uint32_t before = (wid > 0 ? warp_sums[wid - 1] : 0u) + x - v;
+  total = warp_sums[31];
+  __syncthreads();
+  return before;
+}
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
+    select_radix(SelectArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int grp = b * a.Hkv + g;
+  const int L = a.L;
+  const int K = a.kept.kept[grp];
+  const float* sc = a.scores + (size_t)grp * L;
+  int32_t* pm = a.perm + (size_t)grp * L;
+  const int per = (L + kClusterCtas - 1) / kClusterCtas;
+  const int lo = min(L, rank * per);
+  const int hi = min(L, lo + per);
+  const int tid = threadIdx.x;
+
+  __shared__ uint32_t hist[2][256];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t dig_warp[8];
+  __shared__ uint32_t sh_digit, sh_above;
+  __shared__ uint32_t cnt[2];  // this slice's (#key > T, #key == T)
+
+  const bool partial = K < L;
+  uint32_t prefix = 0u, mask = 0u, krem = (uint32_t)K;
+  if (partial) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      uint32_t* h = hist[pass & 1];
+      if (tid < 256) h[tid] = 0u;
+      __syncthreads();
+      for (int i = lo + tid; i < hi; i += kThreads) {
+        const uint32_t key = order_key(sc[i]);
+        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+      }
+      cluster.sync();
+      if (tid < 256) {
+        // Thread t stands for digit 255 - t, so an inclusive scan over t gives
+        // the number of matching keys whose digit is >= 255 - t.
+        uint32_t tot = 0u;
+        for (int r = 0; r < kClusterCtas; ++r) tot += cluster.map_shared_rank(h, r)[255 - tid];
+        const int lane = tid & 31, wid = tid >> 5;
+        uint32_t x = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) dig_warp[wid] = x;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        uint32_t off = 0u;
+        for (int w = 0; w < wid; ++w) off += dig_warp[w];
+        const uint32_t S = off + x;
+        if (S >= krem && S - tot < krem) {
+          sh_digit = 255u - (uint32_t)tid;
+          sh_above = S - tot;
+        }
+      }
+      __syncthreads();
+      prefix |= sh_digit << shift;
+      mask |= 0xFFu << shift;
+      krem -= sh_above;
+    }
+  }
+  const uint32_t T = prefix;
+
+  // Per-slice counts, exchanged over the cluster.
+  if (tid < 2) cnt[tid] = 0u;
+  __syncthreads();
+  if (partial) {
+    uint32_t gt = 0u, eq = 0u;
+    for (int i = lo + tid; i < hi; i += kThreads) {
+      const uint32_t key = order_key(sc[i]);
+      gt += key > T;
+      eq += key == T;
+    }
+    if (gt) atomicAdd(&cnt[0], gt);
+    if (eq) atomicAdd(&cnt[1], eq);
+  }
+  cluster.sync();
+  uint32_t gt_before = 0u, eq_before = 0u;
+  if (partial) {
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t* rc = cluster.map_shared_rank(cnt, r);
+      gt_before += rc[0];
+      eq_before += rc[1];
+    }
+  } else {
+    gt_before = (uint32_t)lo;  // everything is kept: index i lands at i
+  }
+
+  for (int base = lo; base < hi; base += kChunk) {
+    const int i0 = base + tid * kPerThread;
+    uint32_t isgt[kPerThread], iseq[kPerThread];
+    uint32_t ngt = 0u, neq = 0u;
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+      const int i = i0 + e;
+      isgt[e] = 0u;
+      iseq[e] = 0u;
+      if (i < hi) {
+        if (partial) {
+          const uint32_t key = order_key(sc[i]);
+          isgt[e] = key > T;
+          iseq[e] = key == T;
+        } else {
+          isgt[e] = 1u;
+        }
+      }
+      ngt += isgt[e];
+      neq += iseq[e];
+    }
+    uint32_t total;
+    const uint32_t ex = block_exclusive_scan((neq << 16) | ngt, warp_sums, total);
+    uint32_t gb = gt_before + (ex & 0xFFFFu);
+    uint32_t eb = eq_before + (ex >> 16);
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+      const int i = i0 + e;
+      if (i < hi) {
+        const uint32_t S = gb + min(eb, krem);  // kept indices before i
+        const bool keep = isgt[e] || (iseq[e] && eb < krem);
+        const uint32_t dst = keep ? S : (uint32_t)K + (uint32_t)i - S;
+        if (dst < (uint32_t)L) {
+          pm[dst] = i;
+        } else {
+          record_status(a.status, TSA_ERR_DEVICE_BOUNDS);
+        }
+        gb += isgt[e];
+        eb += iseq[e];
+      }
+    }
+    gt_before += total & 0xFFFFu;
+    eq_before += total >> 16;
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
+}  // namespace
+
+cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kept, int32_t* perm,
+                          uint32_t* status, cudaStream_t st) {
+  SelectArgs a;
+  a.scores = scores;
+  a.perm = perm;
+  a.status = status;
+  a.L = d.L;
+  a.Hkv = d.Hkv;
+  a.kept = kept;
+  const dim3 grid(kClusterCtas, d.Hkv, d.B);
+  select_radix<<<grid, kThreads, 0, st>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace tsa

@@ -1,0 +1,284 @@
+// Host entry points of the C ABI declared in include/tsa.h: argument checks,
+// workspace layout, launch planning and the device status word.
+#include <math.h>
+
+#include <atomic>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace tsa {
+
+static std::atomic<uint64_t> g_wait_limit{0};
+
+uint64_t wait_limit() {
+  const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
+  return v ? v : (uint64_t{1} << 24);
+}
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int window_rows_padded(const Dims& d, int window) {
+  const int M = d.G * window;
+  return (M + 63) / 64 * 64;
+}
+
+int score_splits(const Dims& d) {
+  const int ntiles = (d.L + kScoreKeyTile - 1) / kScoreKeyTile;
+  const int groups = d.B * d.Hkv;
+  const int want = (2 * 148 + groups - 1) / groups;
+  int s = want < ntiles ? want : ntiles;
+  s = s < kMaxScoreSplits ? s : kMaxScoreSplits;
+  return s < 1 ? 1 : s;
+}
+
+WsLayout ws_layout(const Dims& d, int window) {
+  WsLayout w;
+  size_t off = 0;
+  w.status = off;
+  off += 256;
+  const size_t n = (size_t)d.B * d.Hkv * d.L;
+  w.scores = off;
+  off += align256(n * sizeof(float));
+  w.perm = off;
+  off += align256(n * sizeof(int32_t));
+  const int Mp = window_rows_padded(d, window);
+  w.part = off;
+  off += align256((size_t)d.B * d.Hkv * kMaxScoreSplits * Mp * 2 * sizeof(float));
+  w.lse = off;
+  off += align256((size_t)d.B * d.Hkv * Mp * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tsa_status check_desc(const tsa_desc* desc, Dims* d) {
+  if (desc == nullptr) return TSA_ERR_INVALID_ARG;
+  if (desc->B < 1 || desc->Hq < 1 || desc->Hkv < 1 || desc->L < 1 || desc->D < 1) return TSA_ERR_INVALID_ARG;
+  if (desc->dtype != TSA_F32 && desc->dtype != TSA_BF16) return TSA_ERR_INVALID_ARG;
+  if (desc->Hq % desc->Hkv != 0) return TSA_ERR_INVALID_ARG;
+  if (!(desc->scale >= 0.f) && !(desc->scale < 0.f)) return TSA_ERR_INVALID_ARG;  // NaN
+  if (desc->D != 64 && desc->D != 128) return TSA_ERR_UNSUPPORTED;
+  const int G = desc->Hq / desc->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return TSA_ERR_UNSUPPORTED;
+  if ((long long)desc->B * desc->Hq * desc->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
+  if ((long long)desc->B * desc->Hkv > kMaxGroups) return TSA_ERR_UNSUPPORTED;
+  d->B = desc->B;
+  d->Hq = desc->Hq;
+  d->Hkv = desc->Hkv;
+  d->L = desc->L;
+  d->D = desc->D;
+  d->G = G;
+  d->dtype = desc->dtype;
+  d->scale = desc->scale > 0.f ? desc->scale : 1.0f / sqrtf((float)desc->D);
+  return TSA_OK;
+}
+
+tsa_status check_window(const Dims& d, int window) {
+  if (window < 1 || window > d.L) return TSA_ERR_INVALID_ARG;
+  if (d.G * window > kMaxWindowRows) return TSA_ERR_UNSUPPORTED;
+  return TSA_OK;
+}
+
+tsa_status load_budgets(const Dims& d, const int32_t* budget_host, Budgets* kb) {
+  if (budget_host == nullptr) return TSA_ERR_INVALID_ARG;
+  for (int i = 0; i < d.B * d.Hkv; ++i) {
+    const int32_t x = budget_host[i];
+    if (x < 1) return TSA_ERR_INVALID_ARG;
+    kb->kept[i] = x < d.L ? x : d.L;
+  }
+  return TSA_OK;
+}
+
+uint32_t* status_word(void* ws) { return static_cast<uint32_t*>(ws); }
+
+template <typename P>
+P* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+tsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSA_OK : TSA_ERR_CUDA; }
+
+tsa_status run_score(const Dims& d, const void* q, const void* k, int window, float* scores, void* ws,
+                     cudaStream_t st) {
+  const WsLayout w = ws_layout(d, window);
+  return cuda_status(launch_score_simt(d, q, k, window, scores, ws_ptr<float>(ws, w.part), status_word(ws), st));
+}
+
+tsa_status run_select(const Dims& d, const float* scores, const Budgets& kb, int32_t* perm, void* ws,
+                      cudaStream_t st) {
+  return cuda_status(launch_select(d, scores, kb, perm, status_word(ws), st));
+}
+
+tsa_status run_attend(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
+                      const Budgets& kb, void* out, void* ws, cudaStream_t st) {
+  tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
+  if (s != TSA_OK) return s;
+  return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), st));
+}
+
+__global__ void debug_wait_kernel(uint32_t* status, const uint32_t* flag, uint64_t limit) {
+  if (threadIdx.x == 0 && !bounded_wait_flag(flag, limit)) record_status(status, TSA_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+cudaError_t launch_debug_wait(uint32_t* status, uint32_t* flag, uint64_t limit, cudaStream_t st) {
+  debug_wait_kernel<<<1, 32, 0, st>>>(status, flag, limit);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace tsa
+
+using namespace tsa;
+
+extern "C" {
+
+size_t tsa_workspace_size(const tsa_desc* desc, int32_t window) {
+  Dims d;
+  if (check_desc(desc, &d) != TSA_OK || check_window(d, window) != TSA_OK) return 0;
+  return ws_layout(d, window).total;
+}
+
+tsa_status tsa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+tsa_status tsa_score(const tsa_desc* desc, const void* q, const void* k, int32_t window, float* scores,
+                     void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if ((s = check_window(d, window)) != TSA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || !aligned16(ws)) return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(d, window).total) return TSA_ERR_WORKSPACE;
+  return run_score(d, q, k, window, scores, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_select(const tsa_desc* desc, const float* scores, const int32_t* budget_host, int32_t* perm,
+                      void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!aligned16(scores) || !aligned16(perm) || !aligned16(ws)) return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return run_select(d, scores, kb, perm, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const void* v, const int32_t* perm,
+                      const int32_t* budget_host, void* out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(perm) || !aligned16(out) || !aligned16(ws))
+    return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_forward(const tsa_desc* desc, const void* q, const void* k, const void* v, int32_t window,
+                       const int32_t* budget_host, float* scores_or_null, int32_t* perm_or_null, void* out,
+                       void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if ((s = check_window(d, window)) != TSA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+    return TSA_ERR_INVALID_ARG;
+  if ((scores_or_null && !aligned16(scores_or_null)) || (perm_or_null && !aligned16(perm_or_null)))
+    return TSA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(d, window);
+  if (ws_bytes < w.total) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  float* scores = scores_or_null ? scores_or_null : ws_ptr<float>(ws, w.scores);
+  int32_t* perm = perm_or_null ? perm_or_null : ws_ptr<int32_t>(ws, w.perm);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = run_score(d, q, k, window, scores, ws, st)) != TSA_OK) return s;
+  if ((s = run_select(d, scores, kb, perm, ws, st)) != TSA_OK) return s;
+  return run_attend(d, q, k, v, perm, kb, out, ws, st);
+}
+
+tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void* k_host, const void* v_host,
+                            int32_t window, const int32_t* budget_host, void* out_host, void* q_dev, void* k_dev,
+                            void* v_dev, void* out_dev, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!q_host || !k_host || !v_host || !out_host) return TSA_ERR_INVALID_ARG;
+  const size_t esz = d.dtype == TSA_F32 ? 4 : 2;
+  const size_t qbytes = (size_t)d.B * d.Hq * d.L * d.D * esz;
+  const size_t kvbytes = (size_t)d.B * d.Hkv * d.L * d.D * esz;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(out_dev)) return TSA_ERR_INVALID_ARG;
+  if ((s = check_window(d, window)) != TSA_OK) return s;
+  if (ws_bytes < ws_layout(d, window).total) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaMemcpyAsync(k_dev, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaMemcpyAsync(v_dev, v_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+  s = tsa_forward(desc, q_dev, k_dev, v_dev, window, budget_host, nullptr, nullptr, out_dev, ws, ws_bytes, stream);
+  if (s != TSA_OK) return s;
+  if (cudaMemcpyAsync(out_host, out_dev, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TSA_ERR_CUDA;
+  return TSA_OK;
+}
+
+tsa_status tsa_check_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TSA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TSA_ERR_CUDA;
+  switch (word) {
+    case TSA_OK:
+    case TSA_ERR_TIMEOUT:
+    case TSA_ERR_DEVICE_BOUNDS:
+      return static_cast<tsa_status>(word);
+    default:
+      return TSA_ERR_CUDA;
+  }
+}
+
+const char* tsa_status_string(tsa_status s) {
+  switch (s) {
+    case TSA_OK: return "ok";
+    case TSA_ERR_INVALID_ARG: return "invalid argument";
+    case TSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case TSA_ERR_WORKSPACE: return "workspace too small";
+    case TSA_ERR_CUDA: return "CUDA runtime error";
+    case TSA_ERR_TIMEOUT: return "device bounded wait timed out";
+    case TSA_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+  }
+  return "unknown status";
+}
+
+void tsa_debug_set_wait_limit(uint64_t polls) { g_wait_limit.store(polls, std::memory_order_relaxed); }
+
+uint64_t tsa_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream) {
+  if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
+  uint32_t* base = status_word(ws);
+  // base[1] is a header word nothing ever sets.
+  return cuda_status(launch_debug_wait(base, base + 1, wait_limit(), static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

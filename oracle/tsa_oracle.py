@@ -29,7 +29,8 @@ What it computes (each function cites the passage it follows):
   Figure 3 (compress Q/K/V per head, attend, scatter to the full sequence
   layout before the residual add).
 
-All arithmetic is float64 on values widened exactly from the caller's inputs.
+All arithmetic is float64 on values widened exactly from the caller's inputs
+(each function widens only the slices it reads, to bound memory at long L).
 Library primitives (``numpy.matmul``, ``numpy.argsort``) serve as single steps;
 there is no blocking or reordering beyond splitting rows into chunks to bound
 memory, which does not change any row's arithmetic.
@@ -92,10 +93,8 @@ def score(q, k, window: int, scale=None) -> np.ndarray:
     softmax over keys, sum over queries) with the window / causal / grouping
     readings listed in the module docstring.
     """
-    q = _f64(q)
-    k = _f64(k)
-    B, Hq, L, D = q.shape
-    Hkv = k.shape[1]
+    B, Hq, L, D = np.shape(q)
+    Hkv = np.shape(k)[1]
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
     if not 1 <= window <= L:
@@ -108,7 +107,7 @@ def score(q, k, window: int, scale=None) -> np.ndarray:
     for b in range(B):
         for h in range(Hq):
             g = h // G
-            logits = s * (q[b, h, L - window:, :] @ k[b, g].T)  # [window, L]
+            logits = s * (_f64(q[b, h, L - window:, :]) @ _f64(k[b, g]).T)  # [window, L]
             logits = np.where(visible, logits, -np.inf)
             m = logits.max(axis=1, keepdims=True)
             e = np.exp(logits - m)
@@ -155,22 +154,19 @@ def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=No
     positions).  Returns [len(rows), D] float64.  This is Step 3's
     matmul / softmax / matmul on the gathered tensors of Step 2.
     """
-    q = _f64(q)
-    k = _f64(k)
-    v = _f64(v)
-    D = q.shape[-1]
+    D = np.shape(q)[-1]
     s = _scale(D, scale)
     g = h // G
     idx = np.asarray(perm_bg[:K], dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
-    kh = k[b, g, idx]  # [K, D]  gathered keys
-    vh = v[b, g, idx]  # [K, D]  gathered values
+    kh = _f64(k[b, g][idx])  # [K, D]  gathered keys
+    vh = _f64(v[b, g][idx])  # [K, D]  gathered values
     out = np.empty((rows.size, D), dtype=np.float64)
     chunk = max(1, (1 << 22) // max(1, K))
     for c0 in range(0, rows.size, chunk):
         rr = rows[c0:c0 + chunk]
         pq = idx[rr]  # original positions of these queries
-        qh = q[b, h, pq]  # [n, D]  gathered queries
+        qh = _f64(q[b, h][pq])  # [n, D]  gathered queries
         logits = s * (qh @ kh.T)  # [n, K]
         logits = np.where(idx[None, :] <= pq[:, None], logits, -np.inf)
         m = logits.max(axis=1, keepdims=True)
@@ -188,9 +184,8 @@ def attend(q, k, v, perm, budgets, scale=None) -> np.ndarray:
     perm[b, g, i]; every dropped position holds 0 (Step 2's
     ``scatter_attention_output`` starts from a zero tensor).
     """
-    q = _f64(q)
-    B, Hq, L, D = q.shape
-    Hkv = np.asarray(k).shape[1]
+    B, Hq, L, D = np.shape(q)
+    Hkv = np.shape(k)[1]
     G = Hq // Hkv
     kept = clamp_budgets(budgets, L)
     perm = np.asarray(perm, dtype=np.int64)
