@@ -49,6 +49,8 @@ cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kep
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
                                cudaStream_t st);
+cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
+                             const Budgets& kept, void* out, uint32_t* status, cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
 cudaError_t launch_debug_wait(uint32_t* status, uint32_t* flag, uint64_t limit, cudaStream_t st);

@@ -123,6 +123,7 @@ tsa_status run_attend(const Dims& d, const void* q, const void* k, const void* v
                       const Budgets& kb, void* out, void* ws, cudaStream_t st) {
   tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
   if (s != TSA_OK) return s;
+  if (d.dtype == TSA_BF16) return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), st));
   return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), st));
 }
 
