@@ -126,6 +126,24 @@ TSA_API tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k
                       size_t ws_bytes, void* stream);
 
 /*
+ * tsa_score_noalloc -- tsa_score without a caller workspace, for callers that
+ * cannot allocate device memory (for example a plugin inside an engine that
+ * owns all device memory, or a latency-critical loop that must not call
+ * cudaMalloc).  The pages have no counterpart: this is a deployment variant.
+ * Same arguments, layout and result as tsa_score; the per-split partials go
+ * to a fixed 1 MiB array built into the library, reserved on every GPU that
+ * loads it until the process exits.  A shape whose partials exceed 1 MiB
+ * (B*Hkv * splits * G*window rounded up to 64 * 8 bytes, splits =
+ * ceil(296 / (B*Hkv)) capped by ceil(L/64)) returns TSA_ERR_WORKSPACE; the
+ * 32/8-head, window-64 layer fits up to B = 64.  The first call made with a device current looks up the
+ * array's device address; make that first call before any stream capture.
+ * All calls share the array: calls whose kernels overlap on the GPU race and
+ * give wrong scores, so order them on one stream.  Allocates nothing.
+ */
+TSA_API tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const void* k, int32_t window,
+                                     float* scores, void* stream);
+
+/*
  * tsa_forward -- tsa_score, tsa_select and tsa_attend in sequence on `stream`.
  * scores_or_null / perm_or_null: where to keep the intermediates; NULL puts
  * them in the workspace.

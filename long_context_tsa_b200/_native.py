@@ -22,7 +22,7 @@ STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
 EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select", "tsa_attend", "tsa_forward",
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
-            "tsa_debug_wait_never_set", "tsa_debug_launch_count")
+            "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc")
 
 
 class TsaDesc(ctypes.Structure):
@@ -54,6 +54,7 @@ _SIGS = {
     "tsa_debug_set_wait_limit": (None, [ctypes.c_uint64]),
     "tsa_debug_wait_never_set": (ctypes.c_int, [_P, _SZ, _P]),
     "tsa_debug_launch_count": (ctypes.c_uint64, []),
+    "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
 }
 
 
@@ -170,3 +171,10 @@ def tsa_debug_wait_never_set(ws, stream=None):
 def tsa_debug_launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(lib().tsa_debug_launch_count())
+
+
+def tsa_score_noalloc(desc, q, k, window, scores, stream=None):
+    """tsa_score for callers that cannot allocate: no workspace argument; the
+    library's fixed device scratch is used (see include/tsa.h)."""
+    _check(lib().tsa_score_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), int(window), _ptr(scores),
+                                   _stream(stream)), "tsa_score_noalloc")
