@@ -44,6 +44,9 @@ struct Budgets {
 // ---- launchers (return the CUDA error of the launch) ----
 cudaError_t launch_score_simt(const Dims& d, const void* q, const void* k, int window, float* scores,
                               float* part, uint32_t* status, cudaStream_t st);
+cudaError_t launch_score_tc(const Dims& d, const void* q, const void* k, int window, float* scores, float* part,
+                            uint32_t* status, cudaStream_t st);
+int score_tc_splits(const Dims& d);
 cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kept, int32_t* perm,
                           uint32_t* status, cudaStream_t st);
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,

@@ -1,0 +1,413 @@
+// Token scoring on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+//
+// "Token Sparse Attention Long Context" (skill page), Step 1, method
+// "entropy": per-key importance = softmax over keys of the scaled query-key
+// logits, summed over queries -- here over an observation window of the last
+// W queries of the G query heads of each KV group, causally masked.
+//
+// Window rows r = hh*W + w (query head g*G+hh, position L-W+w), padded to
+// Mp = 128 or 256 rows.  Keys stream in tiles of 128 by plain tiled TMA; a
+// CTA owns a contiguous range of key tiles ("split") of one (batch, KV group).
+//   pass 1: S = Qw K^T (window rows on TMEM lanes); per row, over the split's
+//           keys, m = max of x = l*log2(e) and Z = sum 2^(x - m)   -> partials
+//   pass 2: S^T = K Qw^T (keys on TMEM lanes, window rows as columns); with
+//           c_r = m_r + log2 Z_r combined over all splits,
+//           score[j] = sum_r 2^(x_rj - c_r)  -- one thread per key, no
+//           cross-thread reduction.
+// Warp roles (320 threads): warps 0-3 and 4-7 read TMEM (two warpgroups),
+// warp 8 loads (TMA), warp 9 issues tcgen05.mma.  Bounded waits throughout.
+#include <cuda.h>
+#include <math.h>
+
+#include "device_common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+#include "tma_maps.h"
+
+namespace tsa {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTeardownPolls = 1u << 26;
+
+struct ScoreTcParams {
+  float* scores;
+  float* part;  // [groups][nsplit][Mp] x {m (log2 units), Z}
+  uint32_t* status;
+  int Hq, Hkv, L, G, W, M, nsplit;
+  float scale_log2;
+  uint64_t wait_limit;
+};
+
+template <int D, int RH>
+struct SCfg {
+  static constexpr int Mp = 128 * RH;
+  static constexpr int NS = 4;
+  static constexpr int HALVES = D / 64;
+  static constexpr int QW_BYTES = Mp * D * 2;
+  static constexpr int KT_BYTES = 128 * D * 2;
+  static constexpr int OFF_QW = 0;
+  static constexpr int OFF_K = QW_BYTES;
+  static constexpr int OFF_CST = OFF_K + NS * KT_BYTES;  // pass 2: Mp floats
+  static constexpr int OFF_RED = OFF_CST + 256 * 4;      // pass 1, RH == 1: 2 x 128 floats
+  static constexpr int OFF_BAR = OFF_RED + 256 * 4;
+  // barriers: q, full[NS], empty[NS], sfull[2], sfree[2], teardown
+  static constexpr int NBAR = 1 + 2 * NS + 4 + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+};
+
+__device__ __forceinline__ void split_tiles(int s, int nsplit, int ntiles, int& t0, int& t1) {
+  t0 = (int)((long long)ntiles * s / nsplit);
+  t1 = (int)((long long)ntiles * (s + 1) / nsplit);
+}
+
+template <int D, int RH, int PASS>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+             const ScoreTcParams p) {
+  using C = SCfg<D, RH>;
+  constexpr int Mp = C::Mp;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int grp = b * p.Hkv + g;
+  const int L = p.L;
+  const int ntiles = (L + 127) / 128;
+  int t0, t1;
+  split_tiles(split, p.nsplit, ntiles, t0, t1);
+  const int nt = t1 - t0;  // key tiles of this CTA
+  const int j0 = t0 * 128, j1 = min(L, t1 * 128);
+  // Steps: pass 1 with RH == 1 takes two key tiles per step (one per warpgroup);
+  // otherwise one key tile per step.
+  const int per_step = (PASS == 1 && RH == 1) ? 2 : 1;
+  const int nstep = (nt + per_step - 1) / per_step;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_QW, sK = base + C::OFF_K;
+  float* cst = reinterpret_cast<float*>(gbase + C::OFF_CST);
+  float* red = reinterpret_cast<float*>(gbase + C::OFF_RED);
+  const uint32_t bar0 = base + C::OFF_BAR;
+  const uint32_t bar_q = bar0;
+  auto bar_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (1 + C::NS + s); };
+  auto bar_sfull = [&](int i) { return bar0 + 8u * (1 + 2 * C::NS + i); };
+  auto bar_sfree = [&](int i) { return bar0 + 8u * (3 + 2 * C::NS + i); };
+  const uint32_t bar_td = bar0 + 8u * (5 + 2 * C::NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull(i), 1);
+      mbar_init(bar_sfree(i), PASS == 1 ? 256 : 128);
+    }
+    mbar_init(bar_td, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_map(&tmq);
+    tma_prefetch_map(&tmk);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() {
+    record_status(p.status, TSA_ERR_TIMEOUT);
+    *abort_flag = 1;
+  };
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ loads
+    // Window rows: lane l gathers rows 4l..4l+3 of each 128-row block; rows
+    // past M repeat row M-1 (their results are never used).
+    if (lane == 0) mbar_arrive_expect_tx(bar_q, C::QW_BYTES);
+    __syncwarp();
+#pragma unroll
+    for (int rb = 0; rb < RH; ++rb) {
+      int y[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = min(rb * 128 + 4 * lane + e, p.M - 1);
+        const int hh = r / p.W, w = r - hh * p.W;
+        y[e] = (b * p.Hq + g * p.G + hh) * L + (L - p.W + w);
+      }
+#pragma unroll
+      for (int h = 0; h < C::HALVES; ++h)
+        tma_gather4(sQ + h * (Mp * 128) + rb * 16384 + lane * 512, &tmq, bar_q, 64 * h, y[0], y[1], y[2], y[3]);
+    }
+    int issued = 0;
+    if (lane == 0) {
+      const int row0 = (b * p.Hkv + g) * L + j0;
+      for (int u = 0; u < nt; ++u) {
+        if (*abort_flag) break;
+        const int s = u % C::NS;
+        if (u >= C::NS && !mbar_wait(bar_empty(s), ((u / C::NS) - 1) & 1, p.wait_limit, abort_flag)) {
+          fail();
+          break;
+        }
+        mbar_arrive_expect_tx(bar_full(s), C::KT_BYTES);
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_2d(sK + s * C::KT_BYTES + h * 16384, &tmk, bar_full(s), 64 * h, row0 + 128 * u);
+        issued = u + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(bar_q, 0, kTeardownPolls, nullptr);
+        for (int u = (issued > C::NS ? issued - C::NS : 0); u < issued; ++u)
+          mbar_wait(bar_full(u % C::NS), (u / C::NS) & 1, kTeardownPolls, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar_q, 0, p.wait_limit, abort_flag);
+      if (PASS == 1) {
+        constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
+        for (int i = 0; ok && i < nstep; ++i) {
+          const int bf = i & 1;
+          if (i >= 2 && !(ok = mbar_wait(bar_sfree(bf), ((i >> 1) - 1) & 1, p.wait_limit, abort_flag))) break;
+          for (int w = 0; w < 2; ++w) {
+            const int u = RH == 2 ? i : 2 * i + w;
+            if (u >= nt) break;
+            if ((RH == 1 || w == 0) && !(ok = mbar_wait(bar_full(u % C::NS), (u / C::NS) & 1, p.wait_limit,
+                                                         abort_flag)))
+              break;
+            tc_fence_after();
+            const uint32_t qb = sQ + (RH == 2 ? w * 16384 : 0);
+            const uint32_t kb = sK + (u % C::NS) * C::KT_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qoff = (kk >> 2) * (Mp * 128) + (kk & 3) * 32;
+              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ss(tmem + bf * 256 + w * 128, sdesc_sw128(qb + qoff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
+                          IDESC, kk > 0);
+            }
+            if (RH == 1 || w == 1) tc_commit(bar_empty(u % C::NS));
+          }
+          if (!ok) break;
+          tc_commit(bar_sfull(bf));
+        }
+      } else {
+        constexpr uint32_t IDESC = idesc_bf16(128, Mp, 0, 0);
+        for (int u = 0; ok && u < nt; ++u) {
+          const int bf = u & 1;
+          if (u >= 2 && !(ok = mbar_wait(bar_sfree(bf), ((u >> 1) - 1) & 1, p.wait_limit, abort_flag))) break;
+          if (!(ok = mbar_wait(bar_full(u % C::NS), (u / C::NS) & 1, p.wait_limit, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t kb = sK + (u % C::NS) * C::KT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (Mp * 128) + (kk & 3) * 32;
+            mma_bf16_ss(tmem + bf * 256, sdesc_sw128(kb + koff, 16, 1024), sdesc_sw128(sQ + qoff, 16, 1024), IDESC,
+                        kk > 0);
+          }
+          tc_commit(bar_empty(u % C::NS));
+          tc_commit(bar_sfull(bf));
+        }
+      }
+      if (!ok) fail();
+      tc_commit(bar_td);
+      mbar_wait(bar_td, 0, kTeardownPolls, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ TMEM readers
+    const int wg = warp >> 2;
+    const int rl = threadIdx.x & 127;  // TMEM lane of this thread
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    bool ok = true;
+    if (PASS == 1) {
+      const int r = RH == 2 ? wg * 128 + rl : rl;  // window row
+      const int pos = L - p.W + (r % p.W);
+      const bool row_ok = r < p.M;
+      float m = -INFINITY, z = 0.f;
+      for (int i = 0; i < nstep; ++i) {
+        const int bf = i & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (i >> 1) & 1, p.wait_limit, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int u = RH == 2 ? i : 2 * i + wg;
+        float x[128];
+        if (u < nt) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + bf * 256 + wg * 128 + q4 * 32, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[q4 * 32 + e] = __uint_as_float(v[e]) * p.scale_log2;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_sfree(bf));
+        if (u < nt) {
+          const int kbase = j0 + 128 * u;
+          const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this tile
+          if (lim < 128) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              if (e >= lim) x[e] = -INFINITY;
+          }
+          float mt = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 128; ++e) mt = fmaxf(mt, x[e]);
+          if (mt > -INFINITY) {
+            const float mn = fmaxf(m, mt);
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < 128; ++e) s += ex2_approx(x[e] - mn);
+            z = z * ex2_approx(m - mn) + s;
+            m = mn;
+          }
+        }
+      }
+      if (!ok) fail();
+      float* pp = p.part + ((size_t)grp * p.nsplit + split) * Mp * 2;
+      if (RH == 2) {
+        if (ok) {
+          pp[r] = m;
+          pp[Mp + r] = z;
+        }
+      } else {
+        // Both warpgroups saw the same rows on alternate key tiles: merge.  The
+        // named barrier is reached by all 256 threads whatever happened above.
+        if (wg == 1) {
+          red[rl] = m;
+          red[128 + rl] = z;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (wg == 0 && !*abort_flag) {
+          const float m2 = red[rl], z2 = red[128 + rl];
+          const float mn = fmaxf(m, m2);
+          float zz = 0.f;
+          if (mn > -INFINITY)
+            zz = (m > -INFINITY ? z * ex2_approx(m - mn) : 0.f) + (m2 > -INFINITY ? z2 * ex2_approx(m2 - mn) : 0.f);
+          pp[r] = mn;
+          pp[Mp + r] = zz;
+        }
+      }
+    } else {
+      // Combine the row partials of every split: c_r = m_r + log2 Z_r.
+      const float* pbase = p.part + (size_t)grp * p.nsplit * Mp * 2;
+      for (int r = threadIdx.x; r < Mp; r += 256) {
+        float mx = -INFINITY;
+        for (int s = 0; s < p.nsplit; ++s) mx = fmaxf(mx, pbase[(size_t)s * Mp * 2 + r]);
+        float zs = 0.f;
+        if (mx > -INFINITY) {
+          for (int s = 0; s < p.nsplit; ++s) {
+            const float ms = pbase[(size_t)s * Mp * 2 + r];
+            if (ms > -INFINITY) zs += pbase[(size_t)s * Mp * 2 + Mp + r] * ex2_approx(ms - mx);
+          }
+        }
+        cst[r] = (r < p.M && mx > -INFINITY) ? mx + log2f(zs) : INFINITY;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      float* out = p.scores + (size_t)grp * L;
+      for (int u = wg; u < nt; u += 2) {
+        const int bf = u & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (u >> 1) & 1, p.wait_limit, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int key = j0 + 128 * u + rl;
+        const bool tail = key >= L - p.W;  // only the last keys are hidden from some window rows
+        float acc = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < Mp / 32; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + bf * 256 + q4 * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = q4 * 32 + e;
+            float pe = ex2_approx(__uint_as_float(v[e]) * p.scale_log2 - cst[col]);
+            if (tail && key > L - p.W + (col % p.W)) pe = 0.f;
+            acc += pe;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_sfree(bf));
+        if (key < j1) out[key] = acc;
+      }
+      if (!ok) fail();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, int RH>
+cudaError_t launch_passes(const Dims& d, const CUtensorMap& mq, const CUtensorMap& mk, const ScoreTcParams& prm,
+                          cudaStream_t st) {
+  const int smem = SCfg<D, RH>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(score_tc<D, RH, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(score_tc<D, RH, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(prm.nsplit, d.Hkv, d.B);
+  score_tc<D, RH, 1><<<grid, kThreads, smem, st>>>(mq, mk, prm);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  score_tc<D, RH, 2><<<grid, kThreads, smem, st>>>(mq, mk, prm);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int score_tc_splits(const Dims& d) {
+  const int ntiles = (d.L + 127) / 128;
+  const int groups = d.B * d.Hkv;
+  int s = 148 / groups;
+  s = s < 1 ? 1 : s;
+  s = s < ntiles ? s : ntiles;
+  return s < kMaxScoreSplits ? s : kMaxScoreSplits;
+}
+
+cudaError_t launch_score_tc(const Dims& d, const void* q, const void* k, int window, float* scores, float* part,
+                            uint32_t* status, cudaStream_t st) {
+  CUtensorMap mq, mk;
+  if (!make_row_map(&mq, q, (uint64_t)d.B * d.Hq * d.L, d.D) ||
+      !make_tile_map(&mk, k, (uint64_t)d.B * d.Hkv * d.L, d.D, 128))
+    return cudaErrorInvalidValue;
+  ScoreTcParams prm;
+  prm.scores = scores;
+  prm.part = part;
+  prm.status = status;
+  prm.Hq = d.Hq;
+  prm.Hkv = d.Hkv;
+  prm.L = d.L;
+  prm.G = d.G;
+  prm.W = window;
+  prm.M = d.G * window;
+  prm.nsplit = score_tc_splits(d);
+  prm.scale_log2 = d.scale * 1.4426950408889634f;
+  prm.wait_limit = wait_limit();
+  const bool two = prm.M > 128;
+  if (d.D == 64) return two ? launch_passes<64, 2>(d, mq, mk, prm, st) : launch_passes<64, 1>(d, mq, mk, prm, st);
+  return two ? launch_passes<128, 2>(d, mq, mk, prm, st) : launch_passes<128, 1>(d, mq, mk, prm, st);
+}
+
+}  // namespace tsa

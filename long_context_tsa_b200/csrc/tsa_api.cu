@@ -46,7 +46,10 @@ WsLayout ws_layout(const Dims& d, int window) {
   off += align256(n * sizeof(float));
   w.perm = off;
   off += align256(n * sizeof(int32_t));
-  const int Mp = window_rows_padded(d, window);
+  // Partials: the SIMT passes pad the window rows to 64, the tensor-core passes to 128 or 256.
+  const int Mp_simt = window_rows_padded(d, window);
+  const int Mp_tc = d.G * window > 128 ? 256 : 128;
+  const int Mp = Mp_simt > Mp_tc ? Mp_simt : Mp_tc;
   w.part = off;
   off += align256((size_t)d.B * d.Hkv * kMaxScoreSplits * Mp * 2 * sizeof(float));
   w.lse = off;
@@ -111,6 +114,8 @@ tsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSA_OK : TSA_E
 tsa_status run_score(const Dims& d, const void* q, const void* k, int window, float* scores, void* ws,
                      cudaStream_t st) {
   const WsLayout w = ws_layout(d, window);
+  if (d.dtype == TSA_BF16)
+    return cuda_status(launch_score_tc(d, q, k, window, scores, ws_ptr<float>(ws, w.part), status_word(ws), st));
   return cuda_status(launch_score_simt(d, q, k, window, scores, ws_ptr<float>(ws, w.part), status_word(ws), st));
 }
 

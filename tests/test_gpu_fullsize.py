@@ -1,0 +1,72 @@
+"""Parity at the workloads' full sizes, in the launch configuration bench.py times.
+
+Scores are compared in full (the oracle's window scoring is cheap); the
+selection bit for bit on a shared float32 score tensor; attention on a seeded
+sample of kept rows per head (always including the first and last kept rows),
+computed one by one by the oracle on the same permutation; dropped rows in full.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_tsa_b200 import inputs as I
+from oracle import tsa_oracle as O
+
+from .parity_util import Run, assert_dropped_rows_zero, assert_scores_close, compare_attend, host
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+ROWS = 48  # sampled kept rows per query head
+
+
+def _setup(name, seed=0):
+    w = I.WORKLOADS[name]
+    q, k, v = I.make_qkv(w, seed=seed, device=DEV)
+    return w, q, k, v, host(q), host(k), host(v)
+
+
+@pytest.mark.parametrize("name", ["gqa_bf16_L8192", "gqa_bf16_L32768", "gqa_bf16_L131072"])
+def test_forward_full_size(name):
+    w, q, k, v, qn, kn, vn = _setup(name)
+    budgets = w.budgets()
+    r = Run(w, q, k, v)
+    scores, perm, out = r.forward(budgets)  # the path bench.py times
+    ora_s = O.score(qn, kn, w.W)
+    sg = host(scores)
+    assert_scores_close(sg, ora_s)
+    np.testing.assert_allclose(sg.sum(-1), w.W * w.G, rtol=1e-4)
+    # Selection: bit-exact given the same float32 score tensor.
+    np.testing.assert_array_equal(host(perm).astype(np.int64), O.select(sg, budgets))
+    s32 = ora_s.astype(np.float32)
+    ora_perm = O.select(s32, budgets)
+    np.testing.assert_array_equal(host(r.select(torch.from_numpy(s32).to(DEV), budgets)), ora_perm)
+    assert_dropped_rows_zero(out, perm, budgets, w.G)
+    # Attention on the oracle's permutation, sampled rows.
+    out = r.attend(torch.from_numpy(ora_perm.astype(np.int32)).to(DEV), budgets)
+    compare_attend(out, qn, kn, vn, ora_perm, budgets, w.dtype, rows_per_head=ROWS, seed=1)
+    assert_dropped_rows_zero(out, torch.from_numpy(ora_perm).to(DEV), budgets, w.G)
+
+
+def test_ragged_budgets_and_sparsity_sweep_131072():
+    w, q, k, v, qn, kn, vn = _setup("ragged_bf16_L131072")
+    r = Run(w, q, k, v)
+    s32 = O.score(qn, kn, w.W).astype(np.float32)
+    sweeps = [w.budgets(seed=0)] + [[I.sweep_budget(t, w.L)] * (w.B * w.Hkv) for t in I.SWEEP_TAUS]
+    for budgets in sweeps:
+        perm = O.select(s32, budgets)
+        np.testing.assert_array_equal(host(r.select(torch.from_numpy(s32).to(DEV), budgets)), perm)
+        out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
+        compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=16, seed=2)
+        assert_dropped_rows_zero(out, torch.from_numpy(perm).to(DEV), budgets, w.G)
+
+
+def test_dense_keep_all_131072():
+    # K = L through the same library: identity permutation, ordinary causal attention.
+    w, q, k, v, qn, kn, vn = _setup("gqa_bf16_L131072", seed=3)
+    budgets = [w.L] * (w.B * w.Hkv)
+    perm = np.broadcast_to(np.arange(w.L, dtype=np.int64), (w.B, w.Hkv, w.L)).copy()
+    r = Run(w, q, k, v)
+    out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
+    compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=8, seed=3)
