@@ -310,7 +310,8 @@ def main():
     flops = attend_flops(w, budgets)
     achieved = flops / (t_attend / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_simt.cu"])
+    traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
+                                                                       "long_context_tsa_b200/csrc/tc_ptx.cuh"])
 
     e2e = None
     if not args.no_e2e:
@@ -342,13 +343,16 @@ def main():
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
-                   "K_per_kv_head": budgets, "l2": "inputs larger than L2 (q 1.07 GB, k and v 268 MB each)",
+                   "K_per_kv_head": budgets,
+                   "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "
+                          f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each; no flush"),
                    "parallelism": f"{world} independent layers, one per GPU"},
         "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend},
         "attend_tflops": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"bf16_tflops ({peak_src})",
-                     "kernel": "tsa_attend", "traffic_source": traffic_src},
+                     "kernel": "attend_tc (tsa_attend: gather + attention + scatter + zero fill)",
+                     "traffic_source": traffic_src},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,

@@ -14,13 +14,18 @@
 // positions; the causal mask on compacted indices equals the mask on original
 // positions because perm[0:K] is ascending.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3, 4-7  softmax + epilogue of tile 0 / tile 1 (thread = TMEM lane = row)
 //   warp 8          producer: TMA gather4 of Q, K, V rows picked by perm
 //   warp 9          MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
-// Shared memory: Q0 Q1 (128xD), P0 P1 (128x128 bf16), a ring of NS K/V tiles;
-// every tile is K-major with the 128-byte swizzle (V is read MN-major).
+//   warp 10         zero fill: this CTA's share of the group's dropped rows
+//                   perm[K:L] gets +0 in every query head (HBM writes that
+//                   overlap the tensor-bound work of the other warps)
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
+// P_t (bf16) overwrites the first 64 columns of S_t once the softmax has read
+// it, and PV reads it from there (A operand in TMEM).
+// Shared memory: Q0 Q1 (128xD) and a ring of NS K/V tiles, K-major with the
+// 128-byte swizzle (V is read MN-major).
 //
 // Online softmax in base 2 with a lazy rescale: the running max used for P
 // moves only when a row max exceeds it by more than 8 (P <= 2^8), so O is
@@ -32,20 +37,23 @@
 #include "device_common.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
-#include "tma_maps.h"
 
 namespace tsa {
 namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kZeroWarp = 10;
 constexpr uint32_t kTeardownPolls = 1u << 26;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct TcAttendParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
   const int32_t* perm;
   void* out;
   uint32_t* status;
@@ -57,18 +65,19 @@ struct TcAttendParams {
 
 template <int D>
 struct Cfg {
-  static constexpr int NS = D == 128 ? 3 : 4;        // K/V ring stages
-  static constexpr int HALVES = D / 64;              // 64-column (128-byte) swizzle atoms per row
+  static constexpr int NS = D == 128 ? 5 : 8;        // K/V ring stages
   static constexpr int Q_BYTES = 128 * D * 2;
   static constexpr int KV_BYTES = 128 * D * 2;
-  static constexpr int P_BYTES = 128 * 128 * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = 2 * Q_BYTES;
-  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+  static constexpr int OFF_KV = 2 * Q_BYTES;
+  static constexpr int OFF_IDX = OFF_KV + NS * KV_BYTES;  // row tables: Q tiles (2 x 128), K/V tile (128)
+  static constexpr int OFF_BAR = OFF_IDX + 3 * 128 * 4;
   // barriers: q, full[NS], empty[NS], s[2], p[2], o[2], teardown; then tmem slot, abort flag
   static constexpr int NBAR = 1 + 2 * NS + 6 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int CPR = D / 8;    // 16-byte chunks per row
+  static constexpr int RPI = 32 / CPR;  // rows per warp-wide copy instruction
+  static constexpr int DEFER = 2;       // copy groups left in flight before a group is published
   static constexpr uint32_t O_COL0 = 256u;  // S_t lives at column 128 * t
 };
 
@@ -87,9 +96,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    attend_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-              const __grid_constant__ CUtensorMap tmv, const TcAttendParams p) {
+__global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p) {
   using C = Cfg<D>;
   const int bid = blockIdx.x;
   const int c = p.cmax - 1 - bid / p.n_groups;  // heaviest chunks first
@@ -107,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t sQ = base + C::OFF_Q, sP = base + C::OFF_P, sKV = base + C::OFF_KV;
+  const uint32_t sQ = base + C::OFF_Q, sKV = base + C::OFF_KV;
   const uint32_t bar0 = base + C::OFF_BAR;
   const uint32_t bar_q = bar0;
   auto bar_full = [&](int s) { return bar0 + 8u * (1 + s); };
@@ -116,15 +123,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_p = [&](int t) { return bar0 + 8u * (3 + 2 * C::NS + t); };
   auto bar_o = [&](int t) { return bar0 + 8u * (5 + 2 * C::NS + t); };
   const uint32_t bar_td = bar0 + 8u * (7 + 2 * C::NS);
+  int* qtab = reinterpret_cast<int*>(gbase + C::OFF_IDX);          // [2][128] global q rows
+  int* kvtab = reinterpret_cast<int*>(gbase + C::OFF_IDX + 1024);  // [128] global k/v rows
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(bar_q, 32);  // the 32 producer lanes publish their own copies
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar_full(s), 1);
+      mbar_init(bar_full(s), 32);
       mbar_init(bar_empty(s), 1);
     }
     for (int t = 0; t < 2; ++t) {
@@ -140,11 +149,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_map(&tmq);
-    tma_prefetch_map(&tmk);
-    tma_prefetch_map(&tmv);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -157,29 +161,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // Load i (K_0, V_0, K_1, V_1, ...) is fill number i / NS of stage i % NS.
-    int issued = 0;
-    // Q tiles: lane l gathers rows 4l..4l+3 of each tile.
-    if (lane == 0) mbar_arrive_expect_tx(bar_q, 2 * C::Q_BYTES);
-    __syncwarp();
-    for (int t = 0; t < 2; ++t) {
-      int y[4];
+    // Copies are 16-byte cp.async chunks written straight into the 128-byte
+    // swizzled K-major layout the MMA reads; one warp instruction moves RPI
+    // whole rows.  Each tile is one commit group; a group is published (proxy
+    // fence, then an arrive by every lane) once DEFER newer groups are in
+    // flight.  Groups 0 and 1 hold the Q tiles (-> bar_q); group 2 + i holds
+    // load i of the ring (K_0, V_0, K_1, ...; fill i / NS of stage i % NS).
+    // With DEFER < NS the load a slot waits for is always published first.
+    const int my_c = lane % C::CPR, my_r = lane / C::CPR;
+    const uint32_t chunk_off = (uint32_t)(my_c >> 3) * 16384u;
+    auto issue_tile = [&](uint32_t dst, const __nv_bfloat16* src, const int* tab) {
+#pragma unroll 4
+      for (int n = 0; n < 128 / C::RPI; ++n) {
+        const int row = n * C::RPI + my_r;
+        const __nv_bfloat16* g = src + (size_t)tab[row] * D + my_c * 8;
+        cp_async16(dst + chunk_off + row * 128 + ((((uint32_t)my_c & 7u) ^ ((uint32_t)row & 7u)) << 4), g);
+      }
+      cp_async_commit();
+    };
+    auto publish_q = [&]() {  // both Q tiles have landed in shared memory
+      fence_proxy_async_smem();
+      mbar_arrive(bar_q);
+    };
+    auto publish_ring = [&](int r) {  // ring load r has landed
+      fence_proxy_async_smem();
+      mbar_arrive(bar_full(r % C::NS));
+    };
+    // Q rows: lane l fills rows 4l..4l+3 of each tile.
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = 4 * lane + e;
         const int hh = r / p.RP;
         const int pos = min(c * P2 + t * p.RP + (r - hh * p.RP), K - 1);
-        y[e] = (b * p.Hq + g * p.G + hh) * L + load_pos(pm, pos, L, p.status);
+        qtab[t * 128 + r] = (b * p.Hq + g * p.G + hh) * L + load_pos(pm, pos, L, p.status);
       }
-#pragma unroll
-      for (int h = 0; h < C::HALVES; ++h)
-        tma_gather4(sQ + t * C::Q_BYTES + h * 16384 + lane * 512, &tmq, bar_q, 64 * h, y[0], y[1], y[2], y[3]);
-    }
+    __syncwarp();
+    issue_tile(sQ, p.q, qtab);                      // group 0
+    issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);   // group 1
+    int committed = 2;  // groups 0, 1: Q tiles; group 2 + r: ring load r
     const int kv_row0 = (b * p.Hkv + g) * L;
+    int y_next[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y_next[e] = kv_row0 + load_pos(pm, min(4 * lane + e, K - 1), L, p.status);
+    int published = 0;  // ring loads published so far
+    bool q_published = false;
     for (int i = 0; i < 2 * n_kt; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int j = i >> 1;
       const int s = i % C::NS;
+      if ((i & 1) == 0) {  // K_j: tile j's rows become current, fetch tile j+1's indices
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kvtab[4 * lane + e] = y_next[e];
+        __syncwarp();
+        if (j + 1 < n_kt) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            y_next[e] = kv_row0 + load_pos(pm, min((j + 1) * 128 + 4 * lane + e, K - 1), L, p.status);
+        }
+      }
       if (i >= C::NS) {  // wait until load i - NS (same stage) has been consumed
         const bool got = mbar_wait(bar_empty(s), ((i / C::NS) - 1) & 1, p.wait_limit, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
@@ -187,26 +229,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
       }
-      int y[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kidx = min(j * 128 + 4 * lane + e, K - 1);
-        y[e] = kv_row0 + load_pos(pm, kidx, L, p.status);
+      issue_tile(sKV + s * C::KV_BYTES, (i & 1) ? p.v : p.k, kvtab);
+      ++committed;
+      // Publish what has landed, keeping DEFER groups in flight.
+      cp_async_wait<C::DEFER>();  // groups [0, committed - DEFER) have landed
+      if (!q_published && committed - C::DEFER >= 2) {
+        publish_q();
+        q_published = true;
       }
-      if (lane == 0) mbar_arrive_expect_tx(bar_full(s), C::KV_BYTES);
-      __syncwarp();
-      const CUtensorMap* map = (i & 1) ? &tmv : &tmk;
-#pragma unroll
-      for (int h = 0; h < C::HALVES; ++h)
-        tma_gather4(sKV + s * C::KV_BYTES + h * 16384 + lane * 512, map, bar_full(s), 64 * h, y[0], y[1], y[2], y[3]);
-      issued = i + 1;
+      while (2 + published < committed - C::DEFER) publish_ring(published++);
     }
-    // Drain after an abort: wait for the copies this warp issued (a fixed limit,
-    // independent of the debug wait limit) before the CTA can exit.
-    if (*abort_flag) {
-      mbar_wait(bar_q, 0, kTeardownPolls, nullptr);
-      for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i)
-        mbar_wait(bar_full(i % C::NS), (i / C::NS) & 1, kTeardownPolls, nullptr);
+    cp_async_wait_all();
+    if (!q_published) publish_q();
+    while (2 + published < committed) publish_ring(published++);
+  } else if (warp == kZeroWarp) {
+    // ------------------------------------------------------------ zero fill
+    const int U = L - K;  // dropped rows of this group
+    if (U > 0) {
+      const int nc = (K + P2 - 1) / P2;  // CTAs of this group
+      const int lo = (int)((long long)U * c / nc), hi = (int)((long long)U * (c + 1) / nc);
+      constexpr int CPR = D * 2 / 16;  // 16-byte chunks per row
+      constexpr int RPI = 32 / CPR;    // rows per warp instruction
+      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+      uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)(b * p.Hq + g * p.G) * L * D) +
+                  lane % CPR;
+      const size_t head_stride = (size_t)L * CPR;  // in 16-byte chunks
+      for (int u = lo + lane / CPR; u < hi; u += RPI) {
+        const int pos = pm[K + u];
+        if ((unsigned)pos >= (unsigned)L) {
+          record_status(p.status, TSA_ERR_DEVICE_BOUNDS);
+          continue;
+        }
+        uint4* row = ob + (size_t)pos * CPR;
+        for (int hh = 0; hh < p.G; ++hh) row[hh * head_stride] = zero;
+      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -227,15 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       IDESC_QK, kk > 0);
         }
       };
+      // P_t (bf16, two per column) sits in the first 64 columns of S_t.
       auto pv = [&](int t, int i_v, bool acc0) {
         const uint32_t vbase = sKV + (i_v % C::NS) * C::KV_BYTES;
-        const uint32_t pbase = sP + t * C::P_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + C::O_COL0 + t * D, sdesc_sw128(pbase + aoff, 16, 1024),
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + C::O_COL0 + t * D, tmem + (uint32_t)t * 128u + kk * 8,
                       sdesc_sw128(vbase + kk * 2048, 16384, 1024), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
-        }
       };
       if (ok) ok = wait_load(0);
       if (ok) {
@@ -280,31 +334,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_off + C::O_COL0 + t * D;
     const int hh = r / p.RP;
     const int pos = c * P2 + t * p.RP + (r - hh * p.RP);
-    const uint32_t prow = sP + t * C::P_BYTES + r * 128;
-    const uint32_t sw = (uint32_t)(r & 7);
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tmem_ld32(tS + q4 * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[q4 * 32 + e] = __uint_as_float(v[e]) * p.scale_log2;
-      }
+      uint32_t v[128];
+      tmem_ld128(tS, v);  // the whole S row of this thread, one load
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
       if (nvis < 128) {
 #pragma unroll
         for (int e = 0; e < 128; ++e)
-          if (e >= nvis) x[e] = -INFINITY;
+          if (e >= nvis) v[e] = 0xff800000u;  // -inf
       }
-      float mt = -INFINITY;
+      // Row max of the raw logits (the scale is positive), 8 independent chains.
+      float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 128; ++e) mt = fmaxf(mt, x[e]);
+      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
+#pragma unroll
+      for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
       // Lazy rescale: move the reference max only when the tile max exceeds
       // it by more than the threshold (then alpha = 2^(old - new) rescales l
       // and O; P stays <= 2^threshold otherwise).
@@ -314,21 +365,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m_use = mt;
       }
-      float rs = 0.f;
+      const float neg_m = -m_use;
+      float acc8[8];
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t w4[4];
+      for (int e = 0; e < 8; ++e) acc8[e] = 0.f;
+      uint32_t pk[64];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float p0 = ex2_approx(x[ch * 8 + 2 * e2] - m_use);
-          const float p1 = ex2_approx(x[ch * 8 + 2 * e2 + 1] - m_use);
-          rs += p0 + p1;
-          w4[e2] = pack_bf16(p0, p1);
-        }
-        const uint32_t addr = prow + (ch >> 3) * 16384 + ((((uint32_t)ch & 7u) ^ sw) << 4);
-        st_shared_v4(addr, w4[0], w4[1], w4[2], w4[3]);
+      for (int e2 = 0; e2 < 64; ++e2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * e2]), p.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * e2 + 1]), p.scale_log2, neg_m));
+        acc8[(2 * e2) & 7] += p0;
+        acc8[(2 * e2 + 1) & 7] += p1;
+        pk[e2] = pack_bf16(p0, p1);
       }
-      l += rs;
+      l += ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       // O_t is idle here (the commit that released S_t(j) covers PV(t, j-1)).
       // TMEM access is warp-collective, so the whole warp rescales when any
       // lane needs it (alpha = 1 for the others).
@@ -341,9 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
           tmem_st32(tO + q4 * 32, v);
         }
-        tmem_st_wait();
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();  // P (and a rescaled O) are in TMEM before the MMA warp is told
       tc_fence_before();
       mbar_arrive(bar_p(t));
     }
@@ -389,11 +440,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
                       const Budgets& kept, void* out, uint32_t* status, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  if (!make_row_map(&mq, q, (uint64_t)d.B * d.Hq * d.L, D) || !make_row_map(&mk, k, (uint64_t)d.B * d.Hkv * d.L, D) ||
-      !make_row_map(&mv, v, (uint64_t)d.B * d.Hkv * d.L, D))
-    return cudaErrorInvalidValue;
   TcAttendParams prm;
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k);
+  prm.v = static_cast<const __nv_bfloat16*>(v);
   prm.perm = perm;
   prm.out = out;
   prm.status = status;
@@ -413,7 +463,7 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
   cudaError_t e = cudaFuncSetAttribute(attend_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)prm.cmax * prm.n_groups;
-  attend_tc<D><<<(unsigned)nblk, kThreads, smem, st>>>(mq, mk, mv, prm);
+  attend_tc<D><<<(unsigned)nblk, kThreads, smem, st>>>(prm);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -247,16 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int u = RH == 2 ? i : 2 * i + wg;
-        float x[128];
-        if (u < nt) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + bf * 256 + wg * 128 + q4 * 32, v);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[q4 * 32 + e] = __uint_as_float(v[e]) * p.scale_log2;
-          }
-        }
+        uint32_t v[128];
+        if (u < nt) tmem_ld128(tmem + lane_off + bf * 256 + wg * 128, v);
         tc_fence_before();
         mbar_arrive(bar_sfree(bf));
         if (u < nt) {
@@ -265,17 +257,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lim < 128) {
 #pragma unroll
             for (int e = 0; e < 128; ++e)
-              if (e >= lim) x[e] = -INFINITY;
+              if (e >= lim) v[e] = 0xff800000u;  // -inf
           }
-          float mt = -INFINITY;
+          float mx8[8];
 #pragma unroll
-          for (int e = 0; e < 128; ++e) mt = fmaxf(mt, x[e]);
+          for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
+#pragma unroll
+          for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+          const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
           if (mt > -INFINITY) {
             const float mn = fmaxf(m, mt);
-            float s = 0.f;
+            const float neg = -mn;
+            float s8[8];
 #pragma unroll
-            for (int e = 0; e < 128; ++e) s += ex2_approx(x[e] - mn);
-            z = z * ex2_approx(m - mn) + s;
+            for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 128; ++e) s8[e & 7] += ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, neg));
+            z = z * ex2_approx(m - mn) + (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
             m = mn;
           }
         }
@@ -318,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ms > -INFINITY) zs += pbase[(size_t)s * Mp * 2 + Mp + r] * ex2_approx(ms - mx);
           }
         }
-        cst[r] = (r < p.M && mx > -INFINITY) ? mx + log2f(zs) : INFINITY;
+        cst[r] = (r < p.M && mx > -INFINITY) ? -(mx + log2f(zs)) : -INFINITY;  // -c_r
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");
       float* out = p.scores + (size_t)grp * L;
@@ -328,20 +327,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int key = j0 + 128 * u + rl;
-        const bool tail = key >= L - p.W;  // only the last keys are hidden from some window rows
-        float acc = 0.f;
-#pragma unroll
+        // Only keys >= L-W are hidden from some window rows; decide per warp
+        // (TMEM loads are warp-collective).
+        const bool tail = __any_sync(0xffffffffu, key >= L - p.W);
+        float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
         for (int q4 = 0; q4 < Mp / 32; ++q4) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_off + bf * 256 + q4 * 32, v);
+          const float* nc = cst + q4 * 32;
+          if (!tail) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = q4 * 32 + e;
-            float pe = ex2_approx(__uint_as_float(v[e]) * p.scale_log2 - cst[col]);
-            if (tail && key > L - p.W + (col % p.W)) pe = 0.f;
-            acc += pe;
+            for (int e = 0; e < 32; ++e) acc4[e & 3] += ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, nc[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int col = q4 * 32 + e;
+              const float pe = ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, nc[e]));
+              acc4[e & 3] += (key > L - p.W + (col % p.W)) ? 0.f : pe;
+            }
           }
         }
+        const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
         tc_fence_before();
         mbar_arrive(bar_sfree(bf));
         if (key < j1) out[key] = acc;

@@ -126,9 +126,10 @@ tsa_status run_select(const Dims& d, const float* scores, const Budgets& kb, int
 
 tsa_status run_attend(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
                       const Budgets& kb, void* out, void* ws, cudaStream_t st) {
+  // The tensor-core kernel zero-fills the dropped rows itself.
+  if (d.dtype == TSA_BF16) return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), st));
   tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
   if (s != TSA_OK) return s;
-  if (d.dtype == TSA_BF16) return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), st));
   return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), st));
 }
 
