@@ -14,11 +14,13 @@
 // positions; the causal mask on compacted indices equals the mask on original
 // positions because perm[0:K] is ascending.
 //
-// Warp roles (352 threads):
+// Warp roles (512 threads, four warpgroups, 128 registers per thread):
 //   warps 0-3, 4-7  softmax + epilogue of tile 0 / tile 1 (thread = TMEM lane = row)
-//   warp 8          producer: TMA gather4 of Q, K, V rows picked by perm
-//   warp 9          MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
-//   warp 10         zero fill: this CTA's share of the group's dropped rows
+//   warps 8-11      loads: each warp gathers 32 of the 128 rows of every Q/K/V
+//                   tile with 16-byte cp.async (one warp per SM sub-partition:
+//                   a single warp cannot pull gathered rows fast enough)
+//   warp 12         MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
+//   warps 13-15     zero fill: this CTA's share of the group's dropped rows
 //                   perm[K:L] gets +0 in every query head (HBM writes that
 //                   overlap the tensor-bound work of the other warps)
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
@@ -43,10 +45,13 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 352;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kZeroWarp = 10;
+constexpr int kThreads = 512;        // four warpgroups
+constexpr int kProducerWarp0 = 8;    // warps 8-11: loads
+constexpr int kProducerWarps = 4;
+constexpr int kMmaWarp = 12;
+constexpr int kZeroWarp0 = 13;       // warps 13-15: zero fill
+constexpr int kZeroWarps = 3;
+
 constexpr uint32_t kTeardownPolls = 1u << 26;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -131,9 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 32);  // the 32 producer lanes publish their own copies
+    mbar_init(bar_q, 32 * kProducerWarps);  // every producer lane publishes its own copies
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar_full(s), 32);
+      mbar_init(bar_full(s), 32 * kProducerWarps);
       mbar_init(bar_empty(s), 1);
     }
     for (int t = 0; t < 2; ++t) {
@@ -159,7 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     *abort_flag = 1;
   };
 
-  if (warp == kProducerWarp) {
+  if (warp >= 8) {
+   if (warp < kProducerWarp0 + kProducerWarps) {
     // ------------------------------------------------------------ producer
     // Copies are 16-byte cp.async chunks written straight into the 128-byte
     // swizzled K-major layout the MMA reads; one warp instruction moves RPI
@@ -168,12 +174,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     // flight.  Groups 0 and 1 hold the Q tiles (-> bar_q); group 2 + i holds
     // load i of the ring (K_0, V_0, K_1, ...; fill i / NS of stage i % NS).
     // With DEFER < NS the load a slot waits for is always published first.
+    const int pw = warp - kProducerWarp0;  // this warp owns rows [32 pw, 32 pw + 32) of every tile
     const int my_c = lane % C::CPR, my_r = lane / C::CPR;
     const uint32_t chunk_off = (uint32_t)(my_c >> 3) * 16384u;
     auto issue_tile = [&](uint32_t dst, const __nv_bfloat16* src, const int* tab) {
 #pragma unroll 4
-      for (int n = 0; n < 128 / C::RPI; ++n) {
-        const int row = n * C::RPI + my_r;
+      for (int n = 0; n < 32 / C::RPI; ++n) {
+        const int row = 32 * pw + n * C::RPI + my_r;
         const __nv_bfloat16* g = src + (size_t)tab[row] * D + my_c * 8;
         cp_async16(dst + chunk_off + row * 128 + ((((uint32_t)my_c & 7u) ^ ((uint32_t)row & 7u)) << 4), g);
       }
@@ -187,24 +194,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       fence_proxy_async_smem();
       mbar_arrive(bar_full(r % C::NS));
     };
-    // Q rows: lane l fills rows 4l..4l+3 of each tile.
+    // Row tables: lane l owns row 32 pw + l of each tile (the warp reads only its rows).
+    const int my_row = 32 * pw + lane;
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 4 * lane + e;
-        const int hh = r / p.RP;
-        const int pos = min(c * P2 + t * p.RP + (r - hh * p.RP), K - 1);
-        qtab[t * 128 + r] = (b * p.Hq + g * p.G + hh) * L + load_pos(pm, pos, L, p.status);
-      }
+    for (int t = 0; t < 2; ++t) {
+      const int hh = my_row / p.RP;
+      const int pos = min(c * P2 + t * p.RP + (my_row - hh * p.RP), K - 1);
+      qtab[t * 128 + my_row] = (b * p.Hq + g * p.G + hh) * L + load_pos(pm, pos, L, p.status);
+    }
     __syncwarp();
     issue_tile(sQ, p.q, qtab);                      // group 0
     issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);   // group 1
     int committed = 2;  // groups 0, 1: Q tiles; group 2 + r: ring load r
     const int kv_row0 = (b * p.Hkv + g) * L;
-    int y_next[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y_next[e] = kv_row0 + load_pos(pm, min(4 * lane + e, K - 1), L, p.status);
+    int y_next = kv_row0 + load_pos(pm, min(my_row, K - 1), L, p.status);
     int published = 0;  // ring loads published so far
     bool q_published = false;
     for (int i = 0; i < 2 * n_kt; ++i) {
@@ -213,14 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       const int s = i % C::NS;
       if ((i & 1) == 0) {  // K_j: tile j's rows become current, fetch tile j+1's indices
         __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kvtab[4 * lane + e] = y_next[e];
+        kvtab[my_row] = y_next;
         __syncwarp();
-        if (j + 1 < n_kt) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            y_next[e] = kv_row0 + load_pos(pm, min((j + 1) * 128 + 4 * lane + e, K - 1), L, p.status);
-        }
+        if (j + 1 < n_kt) y_next = kv_row0 + load_pos(pm, min((j + 1) * 128 + my_row, K - 1), L, p.status);
       }
       if (i >= C::NS) {  // wait until load i - NS (same stage) has been consumed
         const bool got = mbar_wait(bar_empty(s), ((i / C::NS) - 1) & 1, p.wait_limit, abort_flag);
@@ -242,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     cp_async_wait_all();
     if (!q_published) publish_q();
     while (2 + published < committed) publish_ring(published++);
-  } else if (warp == kZeroWarp) {
+  } else if (warp >= kZeroWarp0) {
     // ------------------------------------------------------------ zero fill
     const int U = L - K;  // dropped rows of this group
     if (U > 0) {
@@ -254,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)(b * p.Hq + g * p.G) * L * D) +
                   lane % CPR;
       const size_t head_stride = (size_t)L * CPR;  // in 16-byte chunks
-      for (int u = lo + lane / CPR; u < hi; u += RPI) {
+      for (int u = lo + (warp - kZeroWarp0) * RPI + lane / CPR; u < hi; u += RPI * kZeroWarps) {
         const int pos = pm[K + u];
         if ((unsigned)pos >= (unsigned)L) {
           record_status(p.status, TSA_ERR_DEVICE_BOUNDS);
@@ -325,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       mbar_wait(bar_td, 0, kTeardownPolls, nullptr);
     }
     __syncwarp();
+   }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
@@ -340,22 +339,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[128];
-      tmem_ld128(tS, v);  // the whole S row of this thread, one load
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
-      if (nvis < 128) {
+      // Pass 1: row max of the raw logits (the scale is positive), 32 columns at a time.
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (e >= nvis) v[e] = 0xff800000u;  // -inf
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t v[32];
+        tmem_ld32(tS + q4 * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = (q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
+          mx4[e & 3] = fmaxf(mx4[e & 3], x);
+        }
       }
-      // Row max of the raw logits (the scale is positive), 8 independent chains.
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
-#pragma unroll
-      for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
+      const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
       // Lazy rescale: move the reference max only when the tile max exceeds
       // it by more than the threshold (then alpha = 2^(old - new) rescales l
       // and O; P stays <= 2^threshold otherwise).
@@ -366,21 +363,28 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         m_use = mt;
       }
       const float neg_m = -m_use;
-      float acc8[8];
+      // Pass 2: P = 2^(x - m) as bf16 pairs into the first 64 columns of S_t;
+      // chunk q4 writes columns [16 q4, 16 q4 + 16), which pass 2 has already read.
+      float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc8[e] = 0.f;
-      uint32_t pk[64];
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t v[32];
+        tmem_ld32(tS + q4 * 32, v);
+        uint32_t pk[16];
 #pragma unroll
-      for (int e2 = 0; e2 < 64; ++e2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * e2]), p.scale_log2, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * e2 + 1]), p.scale_log2, neg_m));
-        acc8[(2 * e2) & 7] += p0;
-        acc8[(2 * e2 + 1) & 7] += p1;
-        pk[e2] = pack_bf16(p0, p1);
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const int e = 2 * e2;
+          const float x0 = (q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
+          const float x1 = (q4 * 32 + e + 1 < nvis) ? __uint_as_float(v[e + 1]) : -INFINITY;
+          const float p0 = ex2_approx(fmaf(x0, p.scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(x1, p.scale_log2, neg_m));
+          acc4[e & 3] += p0;
+          acc4[(e + 1) & 3] += p1;
+          pk[e2] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + q4 * 16, pk);
       }
-      l += ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      l += (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
       // O_t is idle here (the commit that released S_t(j) covers PV(t, j-1)).
       // TMEM access is warp-collective, so the whole warp rescales when any
       // lane needs it (alpha = 1 for the others).
