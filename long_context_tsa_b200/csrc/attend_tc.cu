@@ -340,55 +340,80 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       if (!ok) break;
       tc_fence_after();
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
-      // Pass 1: row max of the raw logits (the scale is positive), 32 columns at a time.
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tmem_ld32(tS + q4 * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = (q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
-          mx4[e & 3] = fmaxf(mx4[e & 3], x);
-        }
-      }
-      const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
-      // Lazy rescale: move the reference max only when the tile max exceeds
-      // it by more than the threshold (then alpha = 2^(old - new) rescales l
-      // and O; P stays <= 2^threshold otherwise).
-      const bool need = mt > m_use + kRescaleThreshold;
-      const float alpha = need ? ex2_approx(m_use - mt) : 1.f;  // 0 when m_use is -inf
-      if (need) {
-        l *= alpha;
-        m_use = mt;
-      }
-      const float neg_m = -m_use;
-      // Pass 2: P = 2^(x - m) as bf16 pairs into the first 64 columns of S_t;
-      // chunk q4 writes columns [16 q4, 16 q4 + 16), which pass 2 has already read.
+      // Only tiles on the diagonal hide keys from some rows (warp-uniform choice).
+      const bool masked = __any_sync(0xffffffffu, nvis < 128);
+      // One pass against the current reference max: t = x * scale - m, P = 2^t,
+      // kept packed in registers while the largest t is tracked.  If a row's
+      // t exceeds the rescale threshold (always on the first tile), the warp
+      // redoes the tile from S (still intact: P is only written afterwards)
+      // with that row's exact tile max as the new reference.
+      uint32_t pk[64];
       float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+      float tmax4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      auto exp_pass = [&](float neg_m, bool track) {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tmem_ld32(tS + q4 * 32, v);
-        uint32_t pk[16];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tS + q4 * 32, v);
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const int e = 2 * e2;
-          const float x0 = (q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
-          const float x1 = (q4 * 32 + e + 1 < nvis) ? __uint_as_float(v[e + 1]) : -INFINITY;
-          const float p0 = ex2_approx(fmaf(x0, p.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(x1, p.scale_log2, neg_m));
-          acc4[e & 3] += p0;
-          acc4[(e + 1) & 3] += p1;
-          pk[e2] = pack_bf16(p0, p1);
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int e = 2 * e2;
+            float x0 = __uint_as_float(v[e]), x1 = __uint_as_float(v[e + 1]);
+            if (masked) {
+              x0 = (q4 * 32 + e < nvis) ? x0 : -INFINITY;
+              x1 = (q4 * 32 + e + 1 < nvis) ? x1 : -INFINITY;
+            }
+            const float t0 = fmaf(x0, p.scale_log2, neg_m);
+            const float t1 = fmaf(x1, p.scale_log2, neg_m);
+            if (track) {
+              tmax4[e & 3] = fmaxf(tmax4[e & 3], t0);
+              tmax4[(e + 1) & 3] = fmaxf(tmax4[(e + 1) & 3], t1);
+            }
+            const float p0 = ex2_approx(t0);
+            const float p1 = ex2_approx(t1);
+            acc4[e & 3] += p0;
+            acc4[(e + 1) & 3] += p1;
+            pk[q4 * 16 + e2] = pack_bf16(p0, p1);
+          }
         }
-        tmem_st16(tS + q4 * 16, pk);
+      };
+      float alpha = 1.f;
+      bool need = true;
+      if (j > 0) {
+        exp_pass(-m_use, true);
+        need = fmaxf(fmaxf(tmax4[0], tmax4[1]), fmaxf(tmax4[2], tmax4[3])) > kRescaleThreshold;
       }
-      l += (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+      const bool redo = __any_sync(0xffffffffu, need);
+      if (redo) {
+        // Exact tile max of the raw logits (the scale is positive).
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tS + q4 * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = (!masked || q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
+            mx4[e & 3] = fmaxf(mx4[e & 3], x);
+          }
+        }
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+        if (need) {
+          alpha = ex2_approx(m_use - mt);  // 0 when m_use is -inf
+          m_use = mt;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc4[e] = 0.f;
+        exp_pass(-m_use, false);
+      }
+      l = l * alpha + ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+      // P (bf16 pairs) into the first 64 columns of S_t.
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_st16(tS + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q4 * 16]));
       // O_t is idle here (the commit that released S_t(j) covers PV(t, j-1)).
       // TMEM access is warp-collective, so the whole warp rescales when any
       // lane needs it (alpha = 1 for the others).
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > 0 && redo) {
 #pragma unroll
         for (int q4 = 0; q4 < D / 32; ++q4) {
           uint32_t v[32];
