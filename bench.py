@@ -57,6 +57,25 @@ def attend_flops(w, budgets) -> float:
     return total
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own independent layer (weak scaling): inputs seeded by rank."""
+    return rank
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings (the job is as slow as its slowest rank)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's tokens over the (max-over-ranks) step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -243,7 +262,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
 
-    q, k, v = I.make_qkv(w, seed=rank, device=dev)
+    q, k, v = I.make_qkv(w, seed=rank_seed(rank), device=dev)
     desc = T.desc_for(q, k)
     ws = T.alloc_workspace(desc, w.W, device=dev)
     scores = torch.empty((w.B, w.Hkv, w.L), dtype=torch.float32, device=dev)
@@ -298,13 +317,10 @@ def main():
     t_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     t_attend = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    if dist is not None:
-        t = torch.tensor([total_ms, t_attend], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, t_attend = float(t[0]), float(t[1])
+    total_ms, t_attend = max_over_ranks([total_ms, t_attend], dist, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.B * w.L
-    value = world * tokens / (ms_per_step / 1e3)
+    value = job_tokens_per_s(world, tokens, ms_per_step)
 
     peaks, peak_src = load_peaks()
     flops = attend_flops(w, budgets)
@@ -382,17 +398,13 @@ def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist):
         T.tsa_forward_host(desc, qh, kh, vh, w.W, budgets, oh, qd, kd, vd, od, ws)
     e.record(stream)
     torch.cuda.synchronize(dev)
-    ms = s.elapsed_time(e) / steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    ms = max_over_ranks([s.elapsed_time(e) / steps], dist, dev)[0]
     st = T.tsa_check_status(ws)
     if st != 0:
         raise RuntimeError(f"device status after e2e: {T.tsa_status_string(st)}")
     world = dist.get_world_size() if dist is not None else 1
     nb = lambda t: t.numel() * t.element_size()  # noqa: E731
-    return {"value": world * w.B * w.L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
+    return {"value": job_tokens_per_s(world, w.B * w.L, ms), "unit": "tokens/s", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
             "d2h_bytes_per_step": nb(q), "ms_per_step": ms, "steps": steps}
 
 
