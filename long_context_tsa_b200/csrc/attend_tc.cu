@@ -53,7 +53,8 @@ constexpr int kZeroWarp0 = 13;       // warps 13-15: zero fill
 constexpr int kZeroWarps = 3;
 
 constexpr uint32_t kTeardownPolls = 1u << 26;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kRescaleBound = 256.0f;     // 2^kRescaleThreshold: the largest P kept without a rescale
 
 struct TcAttendParams {
   const __nv_bfloat16* q;
@@ -342,78 +343,119 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
       // Only tiles on the diagonal hide keys from some rows (warp-uniform choice).
       const bool masked = __any_sync(0xffffffffu, nvis < 128);
-      // One pass against the current reference max: t = x * scale - m, P = 2^t,
-      // kept packed in registers while the largest t is tracked.  If a row's
-      // t exceeds the rescale threshold (always on the first tile), the warp
-      // redoes the tile from S (still intact: P is only written afterwards)
-      // with that row's exact tile max as the new reference.
-      uint32_t pk[64];
-      float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-      float tmax4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      auto exp_pass = [&](float neg_m, bool track) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t v[32];
-          tmem_ld32(tS + q4 * 32, v);
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const int e = 2 * e2;
-            float x0 = __uint_as_float(v[e]), x1 = __uint_as_float(v[e + 1]);
-            if (masked) {
-              x0 = (q4 * 32 + e < nvis) ? x0 : -INFINITY;
-              x1 = (q4 * 32 + e + 1 < nvis) ? x1 : -INFINITY;
-            }
-            const float t0 = fmaf(x0, p.scale_log2, neg_m);
-            const float t1 = fmaf(x1, p.scale_log2, neg_m);
-            if (track) {
-              tmax4[e & 3] = fmaxf(tmax4[e & 3], t0);
-              tmax4[(e + 1) & 3] = fmaxf(tmax4[(e + 1) & 3], t1);
-            }
-            const float p0 = ex2_approx(t0);
-            const float p1 = ex2_approx(t1);
-            acc4[e & 3] += p0;
-            acc4[(e + 1) & 3] += p1;
-            pk[q4 * 16 + e2] = pack_bf16(p0, p1);
-          }
-        }
+      // Fast path (tiles after the first): one pass per 32-column chunk against the
+      // current reference max m, t = x * scale - m, P = 2^t written to TMEM at
+      // once (bf16 pairs over S columns [16 q, 16 q + 16), which were already
+      // read).  A chunk where some row has t > threshold (warp vote) switches the
+      // warp to the exact path: the new reference is that row's exact max over the
+      // unread chunks (the written ones had t <= threshold), the written P chunks
+      // are rescaled in TMEM by alpha = 2^(m - m_new) <= 2^-threshold, and the rest
+      // of the row is computed against m_new.  The first tile always takes the
+      // exact two-pass path.
+      const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+      uint64_t acc2 = 0ull;  // packed fp32 pair of the running row sum
+      auto xval = [&](const uint32_t* v, int q4, int e) -> float {
+        const float x = __uint_as_float(v[e]);
+        return (!masked || q4 * 32 + e < nvis) ? x : -INFINITY;
       };
       float alpha = 1.f;
-      bool need = true;
+      bool rescaled = false;  // warp-uniform: O must be rescaled by alpha
+      int q_bad = 4;          // first chunk with a violation (4 = none)
       if (j > 0) {
-        exp_pass(-m_use, true);
-        need = fmaxf(fmaxf(tmax4[0], tmax4[1]), fmaxf(tmax4[2], tmax4[3])) > kRescaleThreshold;
-      }
-      const bool redo = __any_sync(0xffffffffu, need);
-      if (redo) {
-        // Exact tile max of the raw logits (the scale is positive).
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const uint64_t negm2 = f2_pack(-m_use, -m_use);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t v[32];
           tmem_ld32(tS + q4 * 32, v);
+          // P of this chunk in registers; its largest value decides (P > 2^threshold
+          // <=> t > threshold) before anything is written.
+          uint32_t pk[16];
+          uint64_t accq[2] = {0ull, 0ull};
+          __nv_bfloat162 pm2[2] = {__floats2bfloat162_rn(0.f, 0.f), __floats2bfloat162_rn(0.f, 0.f)};
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = (!masked || q4 * 32 + e < nvis) ? __uint_as_float(v[e]) : -INFINITY;
-            mx4[e & 3] = fmaxf(mx4[e & 3], x);
+          for (int e2 = 0; e2 < 16; ++e2) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(xval(v, q4, 2 * e2), xval(v, q4, 2 * e2 + 1)), scale2, negm2), t0, t1);
+            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+            accq[e2 & 1] = f2_add(accq[e2 & 1], f2_pack(p0, p1));
+            pk[e2] = pack_bf16(p0, p1);
+            pm2[e2 & 1] = __hmax2(pm2[e2 & 1], *reinterpret_cast<const __nv_bfloat162*>(&pk[e2]));
           }
+          const __nv_bfloat162 pmx = __hmax2(pm2[0], pm2[1]);
+          const float pmax = fmaxf(__bfloat162float(pmx.x), __bfloat162float(pmx.y));
+          if (__any_sync(0xffffffffu, pmax > kRescaleBound)) {
+            q_bad = q4;
+            break;
+          }
+          tmem_st16(tS + q4 * 16, pk);
+          acc2 = f2_add(acc2, f2_add(accq[0], accq[1]));
         }
-        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+      } else {
+        q_bad = 0;
+      }
+      if (q_bad < 4) {
+        // Exact path from chunk q_bad on.  New reference: the exact max of the
+        // unread chunks for rows that exceed the threshold (or every row on the
+        // first tile, where m is -inf).
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int q4 = q_bad; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tS + q4 * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, xval(v, q4, e));
+        }
+        const float mt = mx * p.scale_log2;
+        const bool need = mt > m_use + kRescaleThreshold;  // always true on the first tile
         if (need) {
           alpha = ex2_approx(m_use - mt);  // 0 when m_use is -inf
           m_use = mt;
         }
+        rescaled = j > 0 && __any_sync(0xffffffffu, need);
+        // Written chunks: P *= alpha (they were computed against the old reference).
+        if (rescaled) {
+          float a0, a1;
+          f2_unpack(acc2, a0, a1);
+          acc2 = f2_pack(a0 * alpha, a1 * alpha);
+#pragma unroll 1
+          for (int q4 = 0; q4 < q_bad; ++q4) {
+            uint32_t w[32];
+            tmem_ld32(tS + q4 * 16, w);  // 32 columns: chunks q4 and q4 + 1 of P (16 used)
+            uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc4[e] = 0.f;
-        exp_pass(-m_use, false);
+            for (int e = 0; e < 16; ++e) {
+              const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+              pk[e] = pack_bf16(__bfloat162float(h.x) * alpha, __bfloat162float(h.y) * alpha);
+            }
+            tmem_st16(tS + q4 * 16, pk);
+          }
+        }
+        const uint64_t negm2 = f2_pack(-m_use, -m_use);
+#pragma unroll 1
+        for (int q4 = q_bad; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(tS + q4 * 32, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(xval(v, q4, 2 * e2), xval(v, q4, 2 * e2 + 1)), scale2, negm2), t0, t1);
+            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+            acc2 = f2_add(acc2, f2_pack(p0, p1));
+            pk[e2] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + q4 * 16, pk);
+        }
       }
-      l = l * alpha + ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
-      // P (bf16 pairs) into the first 64 columns of S_t.
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_st16(tS + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q4 * 16]));
+      {
+        float s0, s1;
+        f2_unpack(acc2, s0, s1);
+        l = l * alpha + (s0 + s1);
+      }
       // O_t is idle here (the commit that released S_t(j) covers PV(t, j-1)).
       // TMEM access is warp-collective, so the whole warp rescales when any
       // lane needs it (alpha = 1 for the others).
-      if (j > 0 && redo) {
+      if (rescaled) {
 #pragma unroll
         for (int q4 = 0; q4 < D / 32; ++q4) {
           uint32_t v[32];

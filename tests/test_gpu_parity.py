@@ -171,3 +171,29 @@ def test_edge_shapes():
         w = I.custom(Hq=4, Hkv=2, L=L, D=128, dtype="bf16", W=W, sigma=0.5)
         q, k, v, qn, kn, vn = _inputs(w, seed=L)
         check_forward(w, q, k, v, qn, kn, vn, [Kb, max(1, Kb // 2)])
+
+
+@pytest.mark.parametrize("spikes", [[0], [40], [128 + 40], [128 + 100, 256 + 5], [384 + 70, 640 + 127]])
+def test_attend_logit_spikes_force_rescales(spikes):
+    # A kept key whose logit jumps far above the running row max (q.k = 4 * 40 = 160,
+    # i.e. ~20 in log2 units after the 1/sqrt(128) scale, far above the rescale
+    # threshold of 8) makes every later query row move its softmax reference
+    # mid-tile, including after earlier 32-column chunks of the tile were written.
+    w = I.custom("spikes", Hq=8, Hkv=2, L=900, D=128, dtype="bf16", W=16, sigma=0.3)
+    q, k, v = I.make_qkv(w, seed=7, device="cpu")
+    u = torch.randn(128, generator=torch.Generator().manual_seed(3))
+    u = u / u.norm()
+    q = (q.float() + 4.0 * u).to(torch.bfloat16)  # every query leans on u
+    budgets = [800, 777]
+    perm = O.select(np.random.default_rng(4).random((1, 2, 900)).astype(np.float32), budgets)
+    k = k.float()
+    for g in range(2):
+        for c in spikes:
+            if c < budgets[g]:
+                k[0, g, perm[0, g, c]] += 40.0 * u
+    k = k.to(torch.bfloat16)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    r = Run(w, qd, kd, vd)
+    out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
+    compare_attend(out, host(q), host(k), host(v), perm, budgets, "bf16")
+    assert_dropped_rows_zero(out, torch.from_numpy(perm).to(DEV), budgets, w.G)
