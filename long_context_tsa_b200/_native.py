@@ -178,3 +178,4 @@ def tsa_score_noalloc(desc, q, k, window, scores, stream=None):
     library's fixed device scratch is used (see include/tsa.h)."""
     _check(lib().tsa_score_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), int(window), _ptr(scores),
                                    _stream(stream)), "tsa_score_noalloc")
+

@@ -363,10 +363,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       int q_bad = 4;          // first chunk with a violation (4 = none)
       if (j > 0) {
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
+        // S chunks are double-buffered in registers: the load of chunk q + 1 is in
+        // flight while chunk q is processed.
+        uint32_t va[32], vb[32];
+        tmem_ld32(tS, va);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t v[32];
-          tmem_ld32(tS + q4 * 32, v);
+          uint32_t(&v)[32] = (q4 & 1) ? vb : va;
+          uint32_t(&vn)[32] = (q4 & 1) ? va : vb;
+          if (q4 < 3) tmem_ld32_async(tS + (q4 + 1) * 32, vn);
           // P of this chunk in registers; its largest value decides (P > 2^threshold
           // <=> t > threshold) before anything is written.
           uint32_t pk[16];
@@ -383,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           }
           const __nv_bfloat162 pmx = __hmax2(pm2[0], pm2[1]);
           const float pmax = fmaxf(__bfloat162float(pmx.x), __bfloat162float(pmx.y));
-          if (__any_sync(0xffffffffu, pmax > kRescaleBound)) {
+          const bool bad = __any_sync(0xffffffffu, pmax > kRescaleBound);
+          if (q4 < 3) tmem_wait_ld32(vn);  // no load left in flight, whatever happens next
+          if (bad) {
             q_bad = q4;
             break;
           }

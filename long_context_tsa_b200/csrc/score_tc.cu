@@ -254,29 +254,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u < nt) {
           const int kbase = j0 + 128 * u;
           const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this tile
-          if (lim < 128) {
+          const bool masked = __any_sync(0xffffffffu, lim < 128);
+          if (masked) {
 #pragma unroll
             for (int e = 0; e < 128; ++e)
               if (e >= lim) v[e] = 0xff800000u;  // -inf
           }
-          float mx8[8];
+          // z is kept relative to a per-row reference m: any reference gives the
+          // same m + log2 z.  The first tile with a visible key sets m to its exact
+          // max; later tiles sum 2^(x - m) directly and are redone against their own
+          // max only if the sum leaves a safe range (a key far above m).
+          auto tile_sum = [&](float ref) {
+            const uint64_t negm2 = f2_pack(-ref, -ref), sc2 = f2_pack(p.scale_log2, p.scale_log2);
+            uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
+            for (int e2 = 0; e2 < 64; ++e2) {
+              float t0, t1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, negm2), t0, t1);
+              a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(ex2_approx(t0), ex2_approx(t1)));
+            }
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            f2_unpack(a2[0], s0, s1);
+            f2_unpack(a2[1], s2, s3);
+            f2_unpack(a2[2], s4, s5);
+            f2_unpack(a2[3], s6, s7);
+            return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+          };
+          float st = (m > -INFINITY) ? tile_sum(m) : INFINITY;
+          const bool exact = !(st <= 1.8446744e19f);  // > 2^64, NaN, or no reference yet
+          if (__any_sync(0xffffffffu, exact)) {
+            float mx8[8];
 #pragma unroll
-          for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-          const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
-          if (mt > -INFINITY) {
-            const float mn = fmaxf(m, mt);
-            const float neg = -mn;
-            float s8[8];
+            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s8[e] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 128; ++e) s8[e & 7] += ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, neg));
-            z = z * ex2_approx(m - mn) + (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
-            m = mn;
+            for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
+            if (exact && mt > -INFINITY) {
+              const float mn = fmaxf(m, mt);
+              const float zs = (m > -INFINITY) ? z * ex2_approx(m - mn) : 0.f;
+              m = mn;
+              z = zs;
+            }
+            if (exact) st = (m > -INFINITY) ? tile_sum(m) : 0.f;
           }
+          z += st;
         }
       }
       if (!ok) fail();
@@ -337,8 +359,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tmem + lane_off + bf * 256 + q4 * 32, v);
           const float* nc = cst + q4 * 32;
           if (!tail) {
+            const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+            uint64_t a2[2] = {0ull, 0ull};
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc4[e & 3] += ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, nc[e]));
+            for (int e2 = 0; e2 < 16; ++e2) {
+              const uint64_t c2 = *reinterpret_cast<const uint64_t*>(nc + 2 * e2);  // (-c_r, -c_r+1)
+              float t0, t1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, c2), t0, t1);
+              a2[e2 & 1] = f2_add(a2[e2 & 1], f2_pack(ex2_approx(t0), ex2_approx(t1)));
+            }
+            float s0, s1, s2, s3;
+            f2_unpack(a2[0], s0, s1);
+            f2_unpack(a2[1], s2, s3);
+            acc4[0] += s0;
+            acc4[1] += s1;
+            acc4[2] += s2;
+            acc4[3] += s3;
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {

@@ -281,6 +281,7 @@ void tsa_debug_set_wait_limit(uint64_t polls) { g_wait_limit.store(polls, std::m
 
 uint64_t tsa_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+
 tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
   uint32_t* base = status_word(ws);

@@ -41,3 +41,4 @@ def test_out_of_range_index_is_reported_and_context_survives(dtype):
     assert T.tsa_check_status(r.ws) == N.STATUS["TSA_ERR_DEVICE_BOUNDS"]
     out = r.attend(torch.from_numpy(perm.astype(np.int32)).cuda(), budgets)
     compare_attend(out, host(q), host(k), host(v), perm, budgets, dtype)
+
