@@ -336,9 +336,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     const int pos = c * P2 + t * p.RP + (r - hh * p.RP);
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
+    // The two softmax warpgroups take turns (named barriers 1 and 2): at d = 128
+    // the exponentials of one tile keep MUFU as busy as the MMAs of the other
+    // tile keep the tensor core, so the tiles alternate instead of sharing MUFU.
+    // Every iteration performs its barrier operations whatever happens (also
+    // after a timeout), and the arrive counts match the syncs exactly: tile 0
+    // goes first; tile 1 skips its last arrive.
+    const uint32_t bar_mine = 1u + (uint32_t)t, bar_other = 2u - (uint32_t)t;
+    if (t == 1) named_arrive(1u, 256u);
     for (int j = 0; j < n_kt; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
-      if (!ok) break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
+      named_sync(bar_mine, 256u);
+      if (!ok) {
+        if (!(t == 1 && j == n_kt - 1)) named_arrive(bar_other, 256u);
+        continue;
+      }
       tc_fence_after();
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
       // Only tiles on the diagonal hide keys from some rows (warp-uniform choice).
@@ -475,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       tmem_st_wait();  // P (and a rescaled O) are in TMEM before the MMA warp is told
       tc_fence_before();
       mbar_arrive(bar_p(t));
+      if (!(t == 1 && j == n_kt - 1)) named_arrive(bar_other, 256u);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o(t), 0, p.wait_limit, abort_flag));
     if (!ok) {
