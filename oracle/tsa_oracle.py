@@ -20,6 +20,12 @@ What it computes (each function cites the passage it follows):
   ``TokenScorer.select_top_k`` (``torch.topk``) and Step 3 (K clamped to the
   sequence length).  Reading: ties go to the lower index; the kept indices
   are listed ascending, followed by the dropped indices ascending.
+* ``drift``   -- representation drift between two hidden-state tensors:
+  one minus the mean, over all (batch, position) rows, of the cosine of the
+  two rows after each is divided by max(its L2 norm, eps).  Source: the skill
+  page, Step 4, ``LayerStabilityAnalyzer.compute_representation_drift``
+  (``torch.nn.functional.normalize`` then a dot product per row);
+  ``layer_stable`` is the same class's ``is_layer_stable`` window rule.
 * ``attend``  -- gather the kept rows of Q, K, V, run softmax attention on the
   compressed tensors with a causal mask by original positions, and scatter the
   result back to full length with zeros at dropped rows.  Source: same page,
@@ -53,7 +59,11 @@ __all__ = [
     "select",
     "attend",
     "attend_rows",
+    "attend_accumulate",
     "forward",
+    "row_cosine",
+    "drift",
+    "layer_stable",
 ]
 
 
@@ -199,6 +209,28 @@ def attend(q, k, v, perm, budgets, scale=None) -> np.ndarray:
     return out
 
 
+def attend_accumulate(base, q, k, v, perm, budgets, scale=None) -> np.ndarray:
+    """``base`` [B, Hq, L, D] plus the attention output at the kept rows; dropped rows unchanged.
+
+    The skill page's Step 2 ``scatter_add_attention_output`` adds the compressed
+    attention output into an existing full-length tensor at the selected
+    indices (``full_output[batch, indices] += attention_output``) instead of
+    scattering into zeros.
+    """
+    out = _f64(base).copy()
+    B, Hq, L, D = out.shape
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    kept = clamp_budgets(budgets, L)
+    perm = np.asarray(perm, dtype=np.int64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            K = int(kept[b * Hkv + g])
+            out[b, h, perm[b, g, :K]] += attend_rows(q, k, v, perm[b, g], K, b, h, G, np.arange(K), scale)
+    return out
+
+
 def forward(q, k, v, window: int, budgets, scale=None):
     """Score -> select (on float32-rounded scores) -> attend.  Returns (scores64, perm, out).
 
@@ -209,3 +241,40 @@ def forward(q, k, v, window: int, budgets, scale=None):
     perm = select(sc.astype(np.float32), budgets)
     out = attend(q, k, v, perm, budgets, scale)
     return sc, perm, out
+
+
+# Default of torch.nn.functional.normalize, which the skill page's drift uses.
+NORMALIZE_EPS = 1e-12
+
+
+def row_cosine(h_before, h_after, eps: float = NORMALIZE_EPS) -> np.ndarray:
+    """Per-row similarity of [..., hidden] tensors: <a / max(|a|, eps), b / max(|b|, eps)>.
+
+    The skill page, Step 4, ``compute_representation_drift``: both hidden
+    states are L2-normalised along the hidden dimension (norm clamped below at
+    eps, as ``torch.nn.functional.normalize`` does) and multiplied elementwise,
+    then summed over the hidden dimension.
+    """
+    a = _f64(h_before)
+    b = _f64(h_after)
+    na = np.maximum(np.sqrt(np.sum(a * a, axis=-1)), eps)
+    nb = np.maximum(np.sqrt(np.sum(b * b, axis=-1)), eps)
+    return np.sum((a / na[..., None]) * (b / nb[..., None]), axis=-1)
+
+
+def drift(h_before, h_after, eps: float = NORMALIZE_EPS) -> float:
+    """1 - mean of ``row_cosine`` over every (batch, position) row (skill page, Step 4)."""
+    return float(1.0 - np.mean(row_cosine(h_before, h_after, eps)))
+
+
+def layer_stable(history, window: int = 3, threshold: float = 0.1) -> bool:
+    """Stability rule of the skill page, Step 4, ``is_layer_stable``.
+
+    ``history`` is the list of drifts so far, the newest last.  With fewer than
+    ``window`` entries the layer is not stable; otherwise it is stable when the
+    mean of the newest ``window`` drifts is strictly below ``threshold``.
+    """
+    if len(history) < window:
+        return False
+    recent = [float(x) for x in history[-window:]]
+    return sum(recent) / len(recent) < threshold

@@ -273,3 +273,103 @@ def test_attend_budget_above_length_is_clamped():
     perm = np.broadcast_to(np.arange(L), (B, Hkv, L))
     np.testing.assert_array_equal(O.attend(q, k, v, perm, [10 * L]), O.attend(q, k, v, perm, [L]))
     assert O.clamp_budgets([10 * L, 3], L).tolist() == [L, 3]
+
+
+def test_attend_accumulate_adds_at_kept_rows_only():
+    # Step 2's scatter_add: base + attention at the kept rows; with a zero base it
+    # is exactly the scatter into zeros; dropped rows keep the base bit for bit.
+    B, Hq, Hkv, L, D = 1, 4, 2, 30, 8
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    budgets = [9, 17]
+    perm = O.select(rng.random((B, Hkv, L)), budgets)
+    zero = np.zeros((B, Hq, L, D))
+    np.testing.assert_array_equal(O.attend_accumulate(zero, q, k, v, perm, budgets), O.attend(q, k, v, perm, budgets))
+    base = rng.standard_normal((B, Hq, L, D))
+    acc = O.attend_accumulate(base, q, k, v, perm, budgets)
+    att = O.attend(q, k, v, perm, budgets)
+    for g, K in enumerate(budgets):
+        hs = slice(2 * g, 2 * g + 2)
+        kept, drop = perm[0, g, :K], perm[0, g, K:]
+        np.testing.assert_array_equal(acc[0, hs][:, drop], base[0, hs][:, drop])
+        np.testing.assert_allclose(acc[0, hs][:, kept], base[0, hs][:, kept] + att[0, hs][:, kept], rtol=0, atol=1e-14)
+
+
+# --- representation drift (skill page, Step 4) -------------------------------------------
+
+
+def _rows(seed, shape):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def test_drift_identical_negated_and_rescaled_states():
+    a = _rows(30, (2, 17, 96))
+    assert abs(O.drift(a, a)) <= 1e-15
+    assert abs(O.drift(a, -a) - 2.0) <= 1e-15
+    # Cosine ignores each row's positive scale, however large or small (above eps).
+    s = np.exp(np.random.default_rng(31).uniform(-12, 12, size=(2, 17, 1)))
+    assert abs(O.drift(a, s * a)) <= 1e-14
+    np.testing.assert_allclose(O.row_cosine(a, s * a), 1.0, rtol=0, atol=1e-14)
+
+
+def test_drift_orthogonal_rows_is_one():
+    qm, _ = np.linalg.qr(_rows(32, (64, 64)))
+    a = qm[:, :32].T.reshape(1, 32, 64)  # 32 orthonormal rows
+    b = qm[:, 32:].T.reshape(1, 32, 64)  # orthogonal to every row of a
+    assert abs(O.drift(a, b) - 1.0) <= 1e-14
+
+
+def test_drift_known_angles():
+    # before = e1, after = cos(t) e1 + sin(t) e2: the row cosine is cos(t) exactly.
+    t = np.linspace(0.0, np.pi, 11)
+    a = np.zeros((1, 11, 8))
+    b = np.zeros((1, 11, 8))
+    a[0, :, 0] = 1.0
+    b[0, :, 0] = np.cos(t)
+    b[0, :, 1] = np.sin(t)
+    np.testing.assert_allclose(O.row_cosine(a, b)[0], np.cos(t), rtol=0, atol=1e-15)
+    assert abs(O.drift(a, b) - (1.0 - np.cos(t).mean())) <= 1e-15
+
+
+def test_drift_matches_scipy_cosine_distance():
+    from scipy.spatial.distance import cosine
+    a = _rows(33, (3, 9, 40))
+    b = a + 0.7 * _rows(34, (3, 9, 40))
+    ref = np.mean([cosine(x, y) for x, y in zip(a.reshape(-1, 40), b.reshape(-1, 40))])
+    assert abs(O.drift(a, b) - ref) <= 1e-14
+
+
+def test_drift_mean_weights_every_row_equally():
+    # Batch 0: identical rows (cosine 1); batch 1: negated rows (cosine -1) in 3 of 4 rows.
+    a = _rows(35, (2, 4, 16))
+    b = a.copy()
+    b[1, :3] = -a[1, :3]
+    np.testing.assert_allclose(O.row_cosine(a, b), [[1, 1, 1, 1], [-1, -1, -1, 1]], rtol=0, atol=1e-15)
+    assert abs(O.drift(a, b) - (1.0 - 2.0 / 8.0)) <= 1e-15
+    assert O.drift(a, b) == O.drift(b, a)
+
+
+def test_drift_norm_clamped_at_eps():
+    # torch.nn.functional.normalize divides by max(|x|, 1e-12): a zero row stays zero
+    # (cosine 0) and a row of norm 1e-13 becomes a vector of norm 0.1.
+    a = np.zeros((1, 3, 4))
+    b = np.zeros((1, 3, 4))
+    a[0, 0, 0] = 1e-13
+    b[0, 0, 0] = 1.0
+    b[0, 1, 2] = 5.0  # a[0, 1] is all zeros
+    a[0, 2, 1] = b[0, 2, 1] = 3.0
+    cos = O.row_cosine(a, b)[0]
+    np.testing.assert_allclose(cos, [0.1, 0.0, 1.0], rtol=1e-12, atol=0)
+    ta, tb = torch.from_numpy(a), torch.from_numpy(b)
+    tref = (torch.nn.functional.normalize(ta, dim=-1) * torch.nn.functional.normalize(tb, dim=-1)).sum(-1)
+    np.testing.assert_allclose(cos, tref.numpy()[0], rtol=1e-14, atol=0)
+
+
+def test_layer_stable_window_rule():
+    assert not O.layer_stable([0.01, 0.01])  # fewer drifts than the window
+    assert O.layer_stable([0.9, 0.05, 0.05, 0.05])  # only the newest three count
+    assert not O.layer_stable([0.05, 0.05, 0.05, 0.9])
+    assert not O.layer_stable([0.25, 0.25, 0.25], threshold=0.25)  # strictly below
+    assert O.layer_stable([0.2, 0.3, 0.24], threshold=0.25)  # mean 0.2467
+    assert O.layer_stable([0.9, 0.01], window=1)
