@@ -234,6 +234,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--op", default="forward", choices=["forward", "forward-accumulate", "drift"],
+                    help="forward: score/select/attend (the headline); forward-accumulate: the same with the "
+                         "scatter-add attention into a resident output; drift: the representation-drift pass")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -243,6 +246,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.op == "drift":
+        bench_drift(args, I, world, rank, local)
+        return
     w = I.WORKLOADS[args.workload]
     budgets = w.budgets(seed=0)
 
@@ -269,6 +275,9 @@ def main():
     perm = torch.empty((w.B, w.Hkv, w.L), dtype=torch.int32, device=dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
+    accumulate = args.op == "forward-accumulate"
+    if accumulate:
+        out.normal_()  # the residual the attention output is added into
 
     def step(ev=None):
         if ev is not None:
@@ -279,7 +288,10 @@ def main():
         T.tsa_select(desc, scores, budgets, perm, ws)
         if ev is not None:
             ev[2].record(stream)
-        T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
+        if accumulate:
+            T.tsa_attend_accumulate(desc, q, k, v, perm, budgets, out, ws)
+        else:
+            T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
         if ev is not None:
             ev[3].record(stream)
 
@@ -358,7 +370,7 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+        "config": {"workload": args.workload, "op": args.op, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets,
                    "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "
                           f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each; no flush"),
@@ -371,6 +383,92 @@ def main():
                      "traffic_source": traffic_src},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": launches,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def bench_drift(args, I, world, rank, local):
+    """Device-timed representation-drift pass over one [B, L, hidden] pair per rank (HBM-bound)."""
+    import long_context_tsa_b200 as T
+
+    cfg = I.DRIFT_WORKLOAD
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "the drift pass has no reference arm; its "
+                              "oracle is timed only in the forward op's reference arm"}), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    a, b = I.make_hidden(cfg["B"], cfg["L"], cfg["hidden"], cfg["dtype"], cfg["delta"], seed=rank_seed(rank),
+                         device=dev)
+    ws = T.alloc_drift_workspace(dev)
+    drift = torch.empty(1, dtype=torch.float64, device=dev)
+    rows = cfg["B"] * cfg["L"]
+    row_cos = torch.empty(rows, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        T.tsa_drift(a, b, drift, ws, row_cos=row_cos)
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = T.tsa_debug_launch_count()
+    start.record(stream)
+    for _ in range(args.steps):
+        T.tsa_drift(a, b, drift, ws, row_cos=row_cos)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = T.tsa_debug_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    (total_ms,) = max_over_ranks([start.elapsed_time(end)], dist, dev)
+    value_drift = float(drift.item())
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    ms = total_ms / args.steps
+    nbytes = 2 * a.numel() * a.element_size() + 4 * rows  # both tensors read once, one float per row written
+    achieved = nbytes / (ms / 1e3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    traffic, traffic_src = kernel_traffic("drift", cfg["name"], ["long_context_tsa_b200/csrc/drift.cu"])
+    line = {
+        "metric": "representation-drift rows/s (hidden 4096, bf16)",
+        "value": world * rows / (ms / 1e3),
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg["dtype"],
+        "data": "synthetic",
+        "config": {"workload": cfg["name"], "op": "drift", "B": cfg["B"], "L": cfg["L"], "hidden": cfg["hidden"],
+                   "delta": cfg["delta"], "drift": value_drift,
+                   "l2": f"inputs larger than L2 (126 MB): {nbytes / 1e9:.2f} GB read per step; no flush",
+                   "parallelism": f"{world} independent tensor pairs, one per GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_source": f"hbm_gbs ({peak_src})", "kernel": "drift_kernel",
+                     "traffic_source": traffic_src},
+        "cpu_baseline": None,
+        "e2e": None,
         "clocks": clocks,
         "gpu_launches": launches,
     }
@@ -437,7 +535,7 @@ def run_reference(args, w, budgets, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+        "config": {"workload": args.workload, "op": args.op, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": sample + " per step"},

@@ -144,6 +144,17 @@ TSA_API tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const 
                                      float* scores, void* stream);
 
 /*
+ * tsa_attend_accumulate -- tsa_attend, but scatter-ADD into an existing output
+ * ([P1] Step 2 scatter_add_attention_output, `full_output[b, indices] +=
+ * attention_output`): out[b,h,p_i] += attention row i for the kept rows, in
+ * fp32 then rounded once to the output dtype; dropped rows keep their value.
+ * Same arguments and rules as tsa_attend; `out` is read and written.
+ */
+TSA_API tsa_status tsa_attend_accumulate(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                                         const int32_t* perm, const int32_t* budget_host, void* out, void* ws,
+                                         size_t ws_bytes, void* stream);
+
+/*
  * tsa_forward -- tsa_score, tsa_select and tsa_attend in sequence on `stream`.
  * scores_or_null / perm_or_null: where to keep the intermediates; NULL puts
  * them in the workspace.
@@ -164,6 +175,39 @@ TSA_API tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, co
                             const void* v_host, int32_t window, const int32_t* budget_host,
                             void* out_host, void* q_dev, void* k_dev, void* v_dev, void* out_dev,
                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_drift -- representation drift between two hidden-state tensors
+ * ("Token Sparse Attention Long Context" skill page, Step 4,
+ * LayerStabilityAnalyzer.compute_representation_drift):
+ *     drift = 1 - mean_r < a_r / max(|a_r|, 1e-12), b_r / max(|b_r|, 1e-12) >
+ * over the `rows` rows of h_before (a) and h_after (b), each [rows, hidden]
+ * row-major in `dtype` (TSA_F32 or TSA_BF16), device memory, 16-byte aligned,
+ * with hidden * sizeof(element) a multiple of 16 bytes.  Rows are accumulated
+ * in fp32, the mean in fp64.
+ *   row_cos_or_null: device float[rows] receiving each row's cosine, or NULL.
+ *   drift:           device double[1] receiving the drift (8-byte aligned).
+ *   ws:              device workspace of at least tsa_drift_workspace_size()
+ *                    bytes, 16-byte aligned, owned by the caller; calls on
+ *                    one workspace must be ordered on one stream.
+ * One memset and one kernel launch on `stream`; the call returns after
+ * enqueueing.  TSA_ERR_INVALID_ARG for rows < 1, a bad dtype, hidden, pointer
+ * or alignment; TSA_ERR_WORKSPACE for a short workspace.
+ */
+TSA_API size_t tsa_drift_workspace_size(void);
+TSA_API tsa_status tsa_drift(int64_t rows, int32_t hidden, int32_t dtype, const void* h_before,
+                             const void* h_after, float* row_cos_or_null, double* drift, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * tsa_layer_stable -- the same page's LayerStabilityAnalyzer.is_layer_stable
+ * window rule on host data: *stable = 1 when history (n drifts, newest last,
+ * host memory) holds at least `window` entries and the mean of the newest
+ * `window` is strictly below `threshold`, else 0.  TSA_ERR_INVALID_ARG for
+ * window < 1, n < 0, a NULL `stable`, or a NULL history with n > 0.
+ */
+TSA_API tsa_status tsa_layer_stable(const double* history, int32_t n, int32_t window, double threshold,
+                                    int32_t* stable);
 
 /* Synchronise `stream`, return the device status recorded in `ws` (TSA_OK,
  * TSA_ERR_TIMEOUT or TSA_ERR_DEVICE_BOUNDS) and clear it. */

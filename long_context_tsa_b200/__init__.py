@@ -11,16 +11,21 @@ from ._native import (  # noqa: F401
     TSA_F32,
     TsaDesc,
     TsaError,
+    alloc_drift_workspace,
     alloc_workspace,
     desc_for,
     make_desc,
     tsa_attend,
+    tsa_attend_accumulate,
     tsa_check_status,
     tsa_debug_launch_count,
     tsa_debug_set_wait_limit,
     tsa_debug_wait_never_set,
+    tsa_drift,
+    tsa_drift_workspace_size,
     tsa_forward,
     tsa_forward_host,
+    tsa_layer_stable,
     tsa_score,
     tsa_select,
     tsa_status_string,

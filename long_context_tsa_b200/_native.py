@@ -22,7 +22,8 @@ STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
 EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select", "tsa_attend", "tsa_forward",
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
-            "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc")
+            "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
+            "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable")
 
 
 class TsaDesc(ctypes.Structure):
@@ -55,6 +56,11 @@ _SIGS = {
     "tsa_debug_wait_never_set": (ctypes.c_int, [_P, _SZ, _P]),
     "tsa_debug_launch_count": (ctypes.c_uint64, []),
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
+    "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_drift": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tsa_layer_stable": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), _I32, _I32, ctypes.c_double,
+                                        ctypes.POINTER(ctypes.c_int32)]),
 }
 
 
@@ -138,6 +144,12 @@ def tsa_attend(desc, q, k, v, perm, budgets, out, ws, stream=None):
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "tsa_attend")
 
 
+def tsa_attend_accumulate(desc, q, k, v, perm, budgets, out, ws, stream=None):
+    """out[kept rows] += attention (scatter-add); dropped rows are left as they are."""
+    _check(lib().tsa_attend_accumulate(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
+                                       _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "tsa_attend_accumulate")
+
+
 def tsa_forward(desc, q, k, v, window, budgets, out, ws, scores=None, perm=None, stream=None):
     _check(lib().tsa_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), int(window), _budgets(budgets),
                              _ptr(scores), _ptr(perm), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
@@ -179,3 +191,33 @@ def tsa_score_noalloc(desc, q, k, window, scores, stream=None):
     _check(lib().tsa_score_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), int(window), _ptr(scores),
                                    _stream(stream)), "tsa_score_noalloc")
 
+
+def tsa_drift_workspace_size() -> int:
+    return int(lib().tsa_drift_workspace_size())
+
+
+def alloc_drift_workspace(device="cuda") -> torch.Tensor:
+    return torch.empty(tsa_drift_workspace_size(), dtype=torch.uint8, device=device)
+
+
+def tsa_drift(h_before, h_after, drift, ws, row_cos=None, stream=None):
+    """drift[0] = 1 - mean row cosine of two [..., hidden] tensors (f32 or bf16, contiguous);
+    row_cos (float32, one per row) receives the cosines when given."""
+    if h_before.shape != h_after.shape or h_before.dtype != h_after.dtype:
+        raise ValueError("h_before and h_after must have the same shape and dtype")
+    if not (h_before.is_contiguous() and h_after.is_contiguous()):
+        raise ValueError("hidden states must be contiguous")
+    hidden = int(h_before.shape[-1])
+    rows = h_before.numel() // max(hidden, 1)
+    dtype = TSA_BF16 if h_before.dtype == torch.bfloat16 else TSA_F32 if h_before.dtype == torch.float32 else -1
+    _check(lib().tsa_drift(rows, hidden, dtype, _ptr(h_before), _ptr(h_after), _ptr(row_cos), _ptr(drift),
+                           _ptr(ws), ws.numel(), _stream(stream)), "tsa_drift")
+
+
+def tsa_layer_stable(history, window: int = 3, threshold: float = 0.1) -> bool:
+    """Window stability rule on host drifts (newest last)."""
+    n = len(history)
+    arr = (ctypes.c_double * max(n, 1))(*[float(x) for x in history])
+    out = ctypes.c_int32(0)
+    _check(lib().tsa_layer_stable(arr, n, int(window), float(threshold), ctypes.byref(out)), "tsa_layer_stable")
+    return bool(out.value)

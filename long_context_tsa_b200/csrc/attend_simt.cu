@@ -31,6 +31,7 @@ struct AttendArgs {
   uint32_t* status;
   int Hq, Hkv, L, G;
   float scale;
+  int accumulate;  // 1: out[kept rows] += attention
   Budgets kept;
 };
 
@@ -185,7 +186,11 @@ __global__ void __launch_bounds__(256) attend_simt(AttendArgs a) {
       const size_t p = (size_t)checked_pos(pm, r, L, a.status);
       const float inv = 1.f / l_i[i];
 #pragma unroll
-      for (int dc = 0; dc < DC; ++dc) oh[p * D + tx + 16 * dc] = from_f32<T>(o[i][dc] * inv);
+      for (int dc = 0; dc < DC; ++dc) {
+        T* dst = oh + p * D + tx + 16 * dc;
+        const float val = o[i][dc] * inv;
+        *dst = from_f32<T>(a.accumulate ? to_f32(*dst) + val : val);
+      }
     }
   }
 }
@@ -228,6 +233,7 @@ AttendArgs make_args(const Dims& d, const void* q, const void* k, const void* v,
   a.L = d.L;
   a.G = d.G;
   a.scale = d.scale;
+  a.accumulate = 0;
   a.kept = kept;
   return a;
 }
@@ -266,8 +272,9 @@ void kept_range(const Dims& d, const Budgets& kept, int& mn, int& mx) {
 
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
-                               cudaStream_t st) {
-  const AttendArgs a = make_args(d, q, k, v, perm, kept, out, status);
+                               bool accumulate, cudaStream_t st) {
+  AttendArgs a = make_args(d, q, k, v, perm, kept, out, status);
+  a.accumulate = accumulate ? 1 : 0;
   int mn, mx;
   kept_range(d, kept, mn, mx);
   if (d.dtype == TSA_F32)

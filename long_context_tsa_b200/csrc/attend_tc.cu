@@ -66,6 +66,7 @@ struct TcAttendParams {
   int Hq, Hkv, L, G, RP, n_groups, cmax;
   float scale_log2;
   uint64_t wait_limit;
+  int accumulate;  // 1: out[kept rows] += attention, dropped rows untouched
   Budgets kept;
 };
 
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     while (2 + published < committed) publish_ring(published++);
   } else if (warp >= kZeroWarp0) {
     // ------------------------------------------------------------ zero fill
-    const int U = L - K;  // dropped rows of this group
+    const int U = p.accumulate ? 0 : L - K;  // dropped rows of this group (none to write when accumulating)
     if (U > 0) {
       const int nc = (K + P2 - 1) / P2;  // CTAs of this group
       const int lo = (int)((long long)U * c / nc), hi = (int)((long long)U * (c + 1) / nc);
@@ -506,11 +507,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(v[8 * e + u]) * inv;
+            if (p.accumulate) {  // scatter-add: the row's current value plus the attention output
+              const uint4 old = dst[e];
+              const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&ow[u]);
+                f[2 * u] += __bfloat162float(h.x);
+                f[2 * u + 1] += __bfloat162float(h.y);
+              }
+            }
             uint4 o;
-            o.x = pack_bf16(__uint_as_float(v[8 * e + 0]) * inv, __uint_as_float(v[8 * e + 1]) * inv);
-            o.y = pack_bf16(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv);
-            o.z = pack_bf16(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv);
-            o.w = pack_bf16(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv);
+            o.x = pack_bf16(f[0], f[1]);
+            o.y = pack_bf16(f[2], f[3]);
+            o.z = pack_bf16(f[4], f[5]);
+            o.w = pack_bf16(f[6], f[7]);
             dst[e] = o;
           }
         }
@@ -530,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
 
 template <int D>
 cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                      const Budgets& kept, void* out, uint32_t* status, cudaStream_t st) {
+                      const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st) {
   TcAttendParams prm;
   prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.k = static_cast<const __nv_bfloat16*>(k);
@@ -546,6 +560,7 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
   prm.n_groups = d.B * d.Hkv;
   prm.scale_log2 = d.scale * 1.4426950408889634f;
   prm.wait_limit = wait_limit();
+  prm.accumulate = accumulate ? 1 : 0;
   prm.kept = kept;
   int kmax = 0;
   for (int i = 0; i < prm.n_groups; ++i) kmax = kept.kept[i] > kmax ? kept.kept[i] : kmax;
@@ -562,9 +577,9 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
 }  // namespace
 
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                             const Budgets& kept, void* out, uint32_t* status, cudaStream_t st) {
-  return d.D == 64 ? launch_tc<64>(d, q, k, v, perm, kept, out, status, st)
-                   : launch_tc<128>(d, q, k, v, perm, kept, out, status, st);
+                             const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st) {
+  return d.D == 64 ? launch_tc<64>(d, q, k, v, perm, kept, out, status, accumulate, st)
+                   : launch_tc<128>(d, q, k, v, perm, kept, out, status, accumulate, st);
 }
 
 }  // namespace tsa

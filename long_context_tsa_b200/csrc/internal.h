@@ -51,11 +51,16 @@ cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kep
                           uint32_t* status, cudaStream_t st);
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
-                               cudaStream_t st);
+                               bool accumulate, cudaStream_t st);
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                             const Budgets& kept, void* out, uint32_t* status, cudaStream_t st);
+                             const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
+constexpr int kDriftMaxBlocks = 2048;  // drift partials held in its workspace
+constexpr size_t kDriftWsBytes = 256 + sizeof(double) * kDriftMaxBlocks;
+int drift_grid(int64_t rows);
+cudaError_t launch_drift(int64_t rows, int hidden, int dtype, const void* a, const void* b, float* row_cos,
+                         double* drift, void* ws, cudaStream_t st);
 cudaError_t launch_debug_wait(uint32_t* status, uint32_t* flag, uint64_t limit, cudaStream_t st);
 
 }  // namespace tsa

@@ -125,12 +125,15 @@ tsa_status run_select(const Dims& d, const float* scores, const Budgets& kb, int
 }
 
 tsa_status run_attend(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                      const Budgets& kb, void* out, void* ws, cudaStream_t st) {
-  // The tensor-core kernel zero-fills the dropped rows itself.
-  if (d.dtype == TSA_BF16) return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), st));
-  tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
-  if (s != TSA_OK) return s;
-  return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), st));
+                      const Budgets& kb, void* out, void* ws, cudaStream_t st, bool accumulate = false) {
+  // The tensor-core kernel zero-fills the dropped rows itself (unless accumulating).
+  if (d.dtype == TSA_BF16)
+    return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), accumulate, st));
+  if (!accumulate) {
+    const tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
+    if (s != TSA_OK) return s;
+  }
+  return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), accumulate, st));
 }
 
 __global__ void debug_wait_kernel(uint32_t* status, const uint32_t* flag, uint64_t limit) {
@@ -196,6 +199,46 @@ tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const 
   Budgets kb;
   if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
   return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_attend_accumulate(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                                 const int32_t* perm, const int32_t* budget_host, void* out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(perm) || !aligned16(out) || !aligned16(ws))
+    return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream), true);
+}
+
+size_t tsa_drift_workspace_size(void) { return kDriftWsBytes; }
+
+tsa_status tsa_drift(int64_t rows, int32_t hidden, int32_t dtype, const void* h_before, const void* h_after,
+                     float* row_cos_or_null, double* drift, void* ws, size_t ws_bytes, void* stream) {
+  if (dtype != TSA_F32 && dtype != TSA_BF16) return TSA_ERR_INVALID_ARG;
+  const int64_t elem = dtype == TSA_BF16 ? 2 : 4;
+  if (rows < 1 || hidden < 1 || (int64_t(hidden) * elem) % 16 != 0) return TSA_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 40) / hidden) return TSA_ERR_INVALID_ARG;  // bounds the row offsets
+  if (!aligned16(h_before) || !aligned16(h_after) || !aligned16(ws) || drift == nullptr) return TSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(drift) & 7u) != 0) return TSA_ERR_INVALID_ARG;
+  if (row_cos_or_null && (reinterpret_cast<uintptr_t>(row_cos_or_null) & 3u) != 0) return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kDriftWsBytes) return TSA_ERR_WORKSPACE;
+  return cuda_status(launch_drift(rows, hidden, dtype, h_before, h_after, row_cos_or_null, drift, ws,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+tsa_status tsa_layer_stable(const double* history, int32_t n, int32_t window, double threshold, int32_t* stable) {
+  if (stable == nullptr || window < 1 || n < 0 || (n > 0 && history == nullptr)) return TSA_ERR_INVALID_ARG;
+  *stable = 0;
+  if (n < window) return TSA_OK;
+  double sum = 0.0;
+  for (int32_t i = n - window; i < n; ++i) sum += history[i];
+  *stable = sum / window < threshold ? 1 : 0;
+  return TSA_OK;
 }
 
 tsa_status tsa_forward(const tsa_desc* desc, const void* q, const void* k, const void* v, int32_t window,
@@ -280,7 +323,6 @@ const char* tsa_status_string(tsa_status s) {
 void tsa_debug_set_wait_limit(uint64_t polls) { g_wait_limit.store(polls, std::memory_order_relaxed); }
 
 uint64_t tsa_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
-
 
 tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;

@@ -153,3 +153,36 @@ def make_scores(B: int, Hkv: int, L: int, seed: int = 0, kind: str = "random") -
         e = torch.randint(-149, -120, (B, Hkv, L), generator=g).float()
         return torch.pow(2.0, e)
     raise ValueError(kind)
+
+
+# --- hidden states for the representation-drift metric ------------------------------------
+#
+# Two [B, L, hidden] tensors shaped like a Llama-3-8B layer's residual stream
+# (hidden = 32 heads * 128 = 4096): h_before has N(0, 1) entries times a
+# log-normal per-row scale (exp(N(0, 0.5^2))) and 4 outlier channels at 20x;
+# h_after = h_before + delta * (fresh N(0, 1) noise at the same row scale).
+# Without the outliers the row cosine would be about 1 / sqrt(1 + delta^2);
+# with them the drift for the default delta = 0.3 is about 0.03, below the
+# 0.05-0.1 stability thresholds the skill page recommends.
+
+DRIFT_WORKLOAD = {"name": "drift_bf16_L131072_h4096", "B": 1, "L": 131072, "hidden": 4096, "dtype": "bf16",
+                  "delta": 0.3}
+
+
+def make_hidden(B: int, L: int, hidden: int, dtype: str = "bf16", delta: float = 0.3, seed: int = 0,
+                device: str | torch.device = "cpu", chunk_rows: int = 8192):
+    """Seeded (h_before, h_after), each [B, L, hidden] in ``dtype``; generated in row chunks on ``device``."""
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator(device=device).manual_seed(seed)
+    before = torch.empty((B * L, hidden), dtype=td, device=device)
+    after = torch.empty_like(before)
+    outliers = torch.randperm(hidden, generator=torch.Generator().manual_seed(seed + 1))[:4].to(device)
+    for r0 in range(0, B * L, chunk_rows):
+        n = min(chunk_rows, B * L - r0)
+        scale = torch.exp(0.5 * torch.randn((n, 1), generator=g, device=device))
+        x = torch.randn((n, hidden), generator=g, device=device)
+        x[:, outliers] *= 20.0
+        x *= scale
+        before[r0:r0 + n] = x.to(td)
+        after[r0:r0 + n] = (x + delta * scale * torch.randn((n, hidden), generator=g, device=device)).to(td)
+    return before.view(B, L, hidden), after.view(B, L, hidden)

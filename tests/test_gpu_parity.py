@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 import torch
 
+import long_context_tsa_b200 as T
 from long_context_tsa_b200 import inputs as I
 from oracle import tsa_oracle as O
 
@@ -197,3 +198,29 @@ def test_attend_logit_spikes_force_rescales(spikes):
     out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
     compare_attend(out, host(q), host(k), host(v), perm, budgets, "bf16")
     assert_dropped_rows_zero(out, torch.from_numpy(perm).to(DEV), budgets, w.G)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_attend_accumulate_scatter_adds(w):
+    # Scatter-add into an existing output: kept rows gain their attention row,
+    # dropped rows keep their previous value bit for bit.
+    q, k, v, qn, kn, vn = _inputs(w, seed=8)
+    rng = np.random.default_rng(9)
+    budgets = [int(x) for x in rng.integers(1, w.L + 1, size=w.B * w.Hkv)]
+    perm = O.select(rng.random((w.B, w.Hkv, w.L)).astype(np.float32), budgets)
+    base = torch.randn(q.shape, generator=torch.Generator().manual_seed(10)).to(q.dtype).to(DEV)
+    out = base.clone()
+    r = Run(w, q, k, v)
+    T.tsa_attend_accumulate(r.desc, q, k, v, torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets, out, r.ws)
+    assert r.status() == 0
+    ora = O.attend_accumulate(host(base), qn, kn, vn, perm, budgets)
+    got = host(out)
+    kept = O.clamp_budgets(budgets, w.L)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            g = h // w.G
+            K = int(kept[b * w.Hkv + g])
+            rows = perm[b, g, :K]
+            assert_rows_close(got[b, h, rows], ora[b, h, rows], w.dtype, f"b={b} h={h}")
+            drop = torch.from_numpy(perm[b, g, K:]).to(DEV)
+            assert torch.equal(out[b, h].index_select(0, drop), base[b, h].index_select(0, drop)), (b, h)
