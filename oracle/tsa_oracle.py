@@ -20,6 +20,16 @@ What it computes (each function cites the passage it follows):
   ``TokenScorer.select_top_k`` (``torch.topk``) and Step 3 (K clamped to the
   sequence length).  Reading: ties go to the lower index; the kept indices
   are listed ascending, followed by the dropped indices ascending.
+* ``coverage_budgets`` -- per-KV-head budget from a token coverage tau:
+  the smallest K whose top-K score mass reaches (1 - tau) of the head's total
+  mass.  Source: "Token Sparse Attention: Efficient Long-Context Inference
+  with Interleaved Token Selection" (sciencestack), the summary's dynamic
+  token coverage and Figures 1 and 5 (sparsity set by a coverage tau); the
+  skill page's Architecture Overview ("Selection Threshold" deciding K per
+  head).  Reading (the pages give no formula): the mass of a token is its
+  score, made exact by fixed point -- floor(clamp(s, 0, 256) * 2^S) as an
+  integer, S = 55 - ceil(log2 L) so that a head's total stays below 2^63 --
+  and the dropped mass may be at most floor(double(M) * tau) of the total M.
 * ``drift``   -- representation drift between two hidden-state tensors:
   one minus the mean, over all (batch, position) rows, of the cosine of the
   two rows after each is divided by max(its L2 norm, eps).  Source: the skill
@@ -57,6 +67,9 @@ __all__ = [
     "clamp_budgets",
     "score",
     "select",
+    "coverage_shift",
+    "token_mass",
+    "coverage_budgets",
     "attend",
     "attend_rows",
     "attend_accumulate",
@@ -153,6 +166,54 @@ def select(scores, budgets) -> np.ndarray:
             perm[b, g, :K] = np.sort(order[:K])
             perm[b, g, K:] = np.sort(order[K:])
     return perm
+
+
+def coverage_shift(L: int) -> int:
+    """Fixed-point shift S of the token masses for sequence length L (L * 256 * 2^S <= 2^63)."""
+    return 55 - max(0, math.ceil(math.log2(L)))
+
+
+def token_mass(scores, L: int) -> np.ndarray:
+    """Integer mass floor(clamp(s, 0, 256) * 2^S) of float32 scores, as uint64 (exact).
+
+    NaN counts as 0 (``fmax``); the coverage reading in the module docstring.
+    """
+    s = np.fmin(np.fmax(np.asarray(scores, dtype=np.float32).astype(np.float64), 0.0), 256.0)
+    return np.floor(s * 2.0 ** coverage_shift(L)).astype(np.uint64)
+
+
+def coverage_budgets(scores, tau: float) -> np.ndarray:
+    """Per (b, g) budget K: the fewest top tokens whose mass reaches the coverage target.
+
+    ``scores`` is float32 [B, Hkv, L].  Per head: M = sum of the integer masses,
+    D = floor(double(M) * tau) (the mass that may be dropped), target
+    T = M - D; K is the smallest k >= 1 such that the k tokens ranked first by
+    ``select``'s order (descending score, lower index first on ties) carry
+    mass >= T.  With T <= 0 (tau = 1, or no mass at all) K = 1.  Returns int64
+    [B * Hkv], ordered like the budgets the other functions take.
+    """
+    s = np.asarray(scores, dtype=np.float32)
+    if s.ndim != 3:
+        raise ValueError("scores must be [B, Hkv, L]")
+    if not np.all(np.isfinite(s)):
+        raise ValueError("scores must be finite")
+    if not (0.0 <= tau <= 1.0):
+        raise ValueError("tau must lie in [0, 1]")
+    B, Hkv, L = s.shape
+    out = np.empty(B * Hkv, dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            m = token_mass(s[b, g], L)
+            M = int(m.sum(dtype=np.uint64))
+            D = math.floor(float(M) * tau)
+            T = M - D
+            if T <= 0:
+                out[b * Hkv + g] = 1
+                continue
+            order = np.argsort(-s[b, g].astype(np.float64), kind="stable")
+            prefix = np.cumsum(m[order], dtype=np.uint64)
+            out[b * Hkv + g] = int(np.searchsorted(prefix, np.uint64(T), side="left")) + 1
+    return out
 
 
 def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=None) -> np.ndarray:

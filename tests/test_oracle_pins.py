@@ -373,3 +373,91 @@ def test_layer_stable_window_rule():
     assert not O.layer_stable([0.25, 0.25, 0.25], threshold=0.25)  # strictly below
     assert O.layer_stable([0.2, 0.3, 0.24], threshold=0.25)  # mean 0.2467
     assert O.layer_stable([0.9, 0.01], window=1)
+
+
+# --- coverage-driven budgets ---------------------------------------------------------------
+
+
+def _brute_coverage(svals, tau):
+    """Plain-Python restatement: integer masses, a sorted list, a linear scan."""
+    L = len(svals)
+    S = 55 - max(0, math.ceil(math.log2(L)))
+    mass = [math.floor(min(max(float(x), 0.0), 256.0) * 2 ** S) for x in svals]
+    M = sum(mass)
+    T = M - math.floor(float(M) * tau)
+    if T <= 0:
+        return 1
+    ranked = sorted(range(L), key=lambda i: (-float(svals[i]), i))
+    acc = 0
+    for k, i in enumerate(ranked, start=1):
+        acc += mass[i]
+        if acc >= T:
+            return k
+    raise AssertionError("unreachable: the full set carries the whole mass")
+
+
+def test_coverage_brute_force_tiny():
+    rng = np.random.default_rng(40)
+    for trial in range(400):
+        L = int(rng.integers(1, 13))
+        kind = trial % 4
+        if kind == 0:
+            s = rng.random(L)
+        elif kind == 1:
+            s = rng.integers(0, 3, size=L) / 4.0  # ties and zeros
+        elif kind == 2:
+            s = rng.exponential(size=L) ** 4  # heavy tail
+        else:
+            s = np.zeros(L)
+        s = s.astype(np.float32)
+        tau = float(rng.choice([0.0, 0.005, 0.1, 0.25, 0.5, 0.9, 1.0, rng.random()]))
+        got = O.coverage_budgets(s.reshape(1, 1, L), tau)[0]
+        assert got == _brute_coverage(s, tau), (s, tau)
+
+
+def test_coverage_closed_forms():
+    L = 1000
+    # Equal scores: every token has the same mass m, so K = ceil(T / m).
+    s = np.full((1, 1, L), 0.25, dtype=np.float32)
+    for tau in (0.0, 0.005, 0.3, 0.999):
+        m = math.floor(0.25 * 2 ** O.coverage_shift(L))
+        M = L * m
+        T = M - math.floor(float(M) * tau)
+        assert O.coverage_budgets(s, tau)[0] == -(-T // m)
+    assert O.coverage_budgets(s, 0.0)[0] == L  # no mass may be dropped
+    assert O.coverage_budgets(s, 1.0)[0] == 1  # all of it may
+    # One token carries all the mass: K = 1 whatever tau.
+    d = np.zeros((1, 1, L), dtype=np.float32)
+    d[0, 0, 517] = 3.0
+    for tau in (0.0, 0.5, 1.0):
+        assert O.coverage_budgets(d, tau)[0] == 1
+    # Geometric masses 2^-i at shuffled positions (exact in fixed point):
+    # keeping k tokens covers (2 - 2^(1-k)) / (2 - 2^(1-n)) of the mass.
+    n = 16
+    g = np.zeros((1, 1, n), dtype=np.float32)
+    g[0, 0, np.random.default_rng(41).permutation(n)] = 2.0 ** -np.arange(n)
+    assert O.coverage_budgets(g, 0.5)[0] == 1
+    assert O.coverage_budgets(g, 0.25)[0] == 2
+    assert O.coverage_budgets(g, 0.1)[0] == 4
+    assert O.coverage_budgets(g, 0.0)[0] == n
+
+
+def test_coverage_minimality_and_monotonicity():
+    rng = np.random.default_rng(42)
+    L = 3000
+    s = (rng.exponential(size=(2, 3, L)) ** 3).astype(np.float32)
+    taus = [0.0, 0.001, 0.005, 0.05, 0.2, 0.6, 1.0]
+    ks = np.stack([O.coverage_budgets(s, t) for t in taus])
+    assert np.all(np.diff(ks, axis=0) <= 0)  # more coverage slack never keeps more tokens
+    for t, k in zip(taus, ks):
+        for bg, K in enumerate(k):
+            b, g = divmod(bg, 3)
+            m = O.token_mass(s[b, g], L)
+            M = int(m.sum())
+            T = M - math.floor(float(M) * t)
+            perm = O.select(s[b:b + 1, g:g + 1], [int(K)])[0, 0]
+            top = int(m[perm[:K]].sum())
+            assert top >= T  # K tokens reach the target ...
+            if K > 1:  # ... and the best K - 1 do not
+                best = np.sort(m)[::-1][:K - 1]
+                assert int(best.sum()) < T
