@@ -234,9 +234,12 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="forward", choices=["forward", "forward-accumulate", "drift"],
+    ap.add_argument("--op", default="forward", choices=["forward", "forward-accumulate", "forward-coverage", "drift"],
                     help="forward: score/select/attend (the headline); forward-accumulate: the same with the "
-                         "scatter-add attention into a resident output; drift: the representation-drift pass")
+                         "scatter-add attention into a resident output; forward-coverage: budgets chosen per KV "
+                         "head from the coverage --tau (one device-to-host copy of the budgets per step); drift: "
+                         "the representation-drift pass")
+    ap.add_argument("--tau", type=float, default=0.005, help="token coverage for --op forward-coverage")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -276,16 +279,23 @@ def main():
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
     accumulate = args.op == "forward-accumulate"
+    coverage = args.op == "forward-coverage"
     if accumulate:
         out.normal_()  # the residual the attention output is added into
+    kdev = torch.empty(w.B * w.Hkv, dtype=torch.int32, device=dev)
 
     def step(ev=None):
+        nonlocal budgets
         if ev is not None:
             ev[0].record(stream)
         T.tsa_score(desc, q, k, w.W, scores, ws)
         if ev is not None:
             ev[1].record(stream)
-        T.tsa_select(desc, scores, budgets, perm, ws)
+        if coverage:
+            T.tsa_select_coverage(desc, scores, args.tau, perm, kdev, ws)
+            budgets = kdev.tolist()  # the attention grid is sized from them
+        else:
+            T.tsa_select(desc, scores, budgets, perm, ws)
         if ev is not None:
             ev[2].record(stream)
         if accumulate:
@@ -370,7 +380,8 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "op": args.op, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+        "config": {"workload": args.workload, "op": args.op, "tau": args.tau if args.op == "forward-coverage" else None,
+                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets,
                    "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "
                           f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each; no flush"),

@@ -144,6 +144,22 @@ TSA_API tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const 
                                      float* scores, void* stream);
 
 /*
+ * tsa_select_coverage -- tsa_select with each (b, g) budget chosen from a
+ * token coverage tau in [0, 1] ("Token Sparse Attention: Efficient
+ * Long-Context Inference with Interleaved Token Selection": dynamic token
+ * coverage; Figures 1 and 5).  Each score s has the integer mass
+ * floor(clamp(s, 0, 256) * 2^S), S = 55 - ceil(log2 L) (NaN counts as 0);
+ * with M the head's total and T = M - floor(double(M) * tau), K is the
+ * smallest k >= 1 whose k top-ranked tokens (tsa_select's order) carry mass
+ * >= T (K = 1 when T = 0).  perm is written as by tsa_select with that K, and
+ * budget_dev_out (device int32[B*Hkv], 4-byte aligned) receives the K values.
+ * One kernel launch; returns after enqueueing.  TSA_ERR_INVALID_ARG for tau
+ * outside [0, 1] or NaN and the pointer rules of tsa_select.
+ */
+TSA_API tsa_status tsa_select_coverage(const tsa_desc* desc, const float* scores, double tau, int32_t* perm,
+                                       int32_t* budget_dev_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * tsa_attend_accumulate -- tsa_attend, but scatter-ADD into an existing output
  * ([P1] Step 2 scatter_add_attention_output, `full_output[b, indices] +=
  * attention_output`): out[b,h,p_i] += attention row i for the kept rows, in
@@ -162,6 +178,19 @@ TSA_API tsa_status tsa_attend_accumulate(const tsa_desc* desc, const void* q, co
 TSA_API tsa_status tsa_forward(const tsa_desc* desc, const void* q, const void* k, const void* v,
                        int32_t window, const int32_t* budget_host, float* scores_or_null,
                        int32_t* perm_or_null, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tsa_forward_coverage -- tsa_score, tsa_select_coverage and tsa_attend in
+ * sequence, budgets chosen from the coverage tau.  The attention grid is
+ * sized from the budgets, so the call copies them into budget_host_out (host
+ * int32[B*Hkv]) and SYNCHRONISES `stream` between the selection and the
+ * attention; it returns after enqueueing the attention.  Same buffers and
+ * workspace rule as tsa_forward.
+ */
+TSA_API tsa_status tsa_forward_coverage(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                                        int32_t window, double tau, int32_t* budget_host_out,
+                                        float* scores_or_null, int32_t* perm_or_null, void* out, void* ws,
+                                        size_t ws_bytes, void* stream);
 
 /*
  * tsa_forward_host -- tsa_forward on HOST inputs and output.  q_host/k_host/

@@ -24,10 +24,12 @@ from ._native import (  # noqa: F401
     tsa_drift,
     tsa_drift_workspace_size,
     tsa_forward,
+    tsa_forward_coverage,
     tsa_forward_host,
     tsa_layer_stable,
     tsa_score,
     tsa_select,
+    tsa_select_coverage,
     tsa_status_string,
     tsa_workspace_init,
     tsa_workspace_size,

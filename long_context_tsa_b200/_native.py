@@ -23,7 +23,8 @@ STATUS = {v: k for k, v in STATUS_NAMES.items()}
 EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select", "tsa_attend", "tsa_forward",
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
-            "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable")
+            "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
+            "tsa_select_coverage", "tsa_forward_coverage")
 
 
 class TsaDesc(ctypes.Structure):
@@ -58,6 +59,9 @@ _SIGS = {
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_select_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, ctypes.c_double, _P, _P, _P, _SZ, _P]),
+    "tsa_forward_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P,
+                                            _P, _P, _SZ, _P]),
     "tsa_drift": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_layer_stable": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), _I32, _I32, ctypes.c_double,
                                         ctypes.POINTER(ctypes.c_int32)]),
@@ -221,3 +225,19 @@ def tsa_layer_stable(history, window: int = 3, threshold: float = 0.1) -> bool:
     out = ctypes.c_int32(0)
     _check(lib().tsa_layer_stable(arr, n, int(window), float(threshold), ctypes.byref(out)), "tsa_layer_stable")
     return bool(out.value)
+
+
+def tsa_select_coverage(desc, scores, tau, perm, budgets_out, ws, stream=None):
+    """Top-K per KV head with K chosen from the coverage tau; budgets_out (int32 device) receives K."""
+    _check(lib().tsa_select_coverage(ctypes.byref(desc), _ptr(scores), float(tau), _ptr(perm), _ptr(budgets_out),
+                                     _ptr(ws), ws.numel(), _stream(stream)), "tsa_select_coverage")
+
+
+def tsa_forward_coverage(desc, q, k, v, window, tau, out, ws, scores=None, perm=None, stream=None):
+    """Score, coverage selection and attention; returns the chosen budgets (list of int)."""
+    n = desc.B * desc.Hkv
+    arr = (ctypes.c_int32 * n)()
+    _check(lib().tsa_forward_coverage(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), int(window), float(tau), arr,
+                                      _ptr(scores), _ptr(perm), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "tsa_forward_coverage")
+    return list(arr)

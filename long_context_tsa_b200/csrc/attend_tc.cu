@@ -53,6 +53,7 @@ constexpr int kZeroWarp0 = 13;       // warps 13-15: zero fill
 constexpr int kZeroWarps = 3;
 
 constexpr uint32_t kTeardownPolls = 1u << 26;
+constexpr long long kFusedZeroMinCtas = 2 * 148;  // attention CTAs from which the zero fill is fused
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kRescaleBound = 256.0f;     // 2^kRescaleThreshold: the largest P kept without a rescale
 
@@ -67,6 +68,7 @@ struct TcAttendParams {
   float scale_log2;
   uint64_t wait_limit;
   int accumulate;  // 1: out[kept rows] += attention, dropped rows untouched
+  int zero_fill;   // 1: warps 13-15 write the dropped rows (else a separate kernel did, or none are due)
   Budgets kept;
 };
 
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     while (2 + published < committed) publish_ring(published++);
   } else if (warp >= kZeroWarp0) {
     // ------------------------------------------------------------ zero fill
-    const int U = p.accumulate ? 0 : L - K;  // dropped rows of this group (none to write when accumulating)
+    const int U = p.zero_fill ? L - K : 0;  // dropped rows of this group left to this kernel
     if (U > 0) {
       const int nc = (K + P2 - 1) / P2;  // CTAs of this group
       const int lo = (int)((long long)U * c / nc), hi = (int)((long long)U * (c + 1) / nc);
@@ -565,10 +567,22 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
   int kmax = 0;
   for (int i = 0; i < prm.n_groups; ++i) kmax = kept.kept[i] > kmax ? kept.kept[i] : kmax;
   prm.cmax = (kmax + 2 * prm.RP - 1) / (2 * prm.RP);
+  const long long nblk = (long long)prm.cmax * prm.n_groups;
+  // The fused zero fill spreads the dropped rows over the attention CTAs; with
+  // fewer of those than two per SM (small budgets) a separate full-grid zero
+  // kernel writes them at HBM speed instead.
+  prm.zero_fill = 0;
+  if (!accumulate) {
+    if (nblk >= kFusedZeroMinCtas) {
+      prm.zero_fill = 1;
+    } else {
+      const cudaError_t ez = launch_zero_fill(d, perm, kept, out, status, st);
+      if (ez != cudaSuccess) return ez;
+    }
+  }
   const int smem = Cfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(attend_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long nblk = (long long)prm.cmax * prm.n_groups;
   attend_tc<D><<<(unsigned)nblk, kThreads, smem, st>>>(prm);
   count_launches(1);
   return cudaGetLastError();

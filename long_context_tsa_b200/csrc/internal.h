@@ -26,6 +26,7 @@ struct WsLayout {
   size_t perm;    // [B,Hkv,L] i32 scratch for tsa_forward
   size_t part;    // score partials [B*Hkv][splits][Mp] x {max, sum} f32
   size_t lse;     // combined per-row log-normaliser [B*Hkv][Mp] f32
+  size_t budgets; // [B*Hkv] i32 budgets chosen on the device (coverage mode)
   size_t total;
 };
 
@@ -49,6 +50,8 @@ cudaError_t launch_score_tc(const Dims& d, const void* q, const void* k, int win
 int score_tc_splits(const Dims& d);
 cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kept, int32_t* perm,
                           uint32_t* status, cudaStream_t st);
+cudaError_t launch_select_coverage(const Dims& d, const float* scores, double tau, int32_t* perm, int32_t* k_out,
+                                   uint32_t* status, cudaStream_t st);
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
                                bool accumulate, cudaStream_t st);

@@ -14,6 +14,18 @@
 // memory; each CTA then derives the same digit.  Compaction: the kept position
 // of index i is  #(keys > T before i) + min(#(keys == T before i), ties_left),
 // a block-wide scan per chunk plus the slice offsets exchanged over the cluster.
+//
+// Coverage mode (budgets from a token coverage tau, "Token Sparse Attention:
+// Efficient Long-Context Inference with Interleaved Token Selection", dynamic
+// token coverage, Figures 1 and 5): each score s carries the integer mass
+// floor(clamp(s, 0, 256) * 2^S); the head's total M is summed over the
+// cluster, the target is T = M - floor(double(M) * tau), and K is the fewest
+// top-ranked tokens whose mass reaches T.  The four radix passes then build
+// mass histograms (u64) beside the count histograms and descend to the digit
+// where the mass from the top crosses the remaining target; at the end the
+// key of the K-th token is known, with the count and mass of every key above
+// it, and  K = above + ceil(remaining target / mass of that key).  Integer
+// sums make K independent of the summation order.
 #include <cooperative_groups.h>
 
 #include "device_common.cuh"
@@ -34,8 +46,52 @@ struct SelectArgs {
   int32_t* perm;
   uint32_t* status;
   int L, Hkv;
+  int coverage;       // 1: K from tau (below), 0: K from kept
+  double tau;
+  float mass_scale;   // 2^S
+  int32_t* k_out;     // [B * Hkv] chosen K (coverage mode), or null
   Budgets kept;
 };
+
+__device__ __forceinline__ uint64_t token_mass(float s, float mass_scale) {
+  // fmaxf drops NaN; scaling by a power of two is exact; truncation is floor here.
+  return __float2ull_rz(fminf(fmaxf(s, 0.f), 256.f) * mass_scale);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Inclusive scan over the 256 digit threads (tid < 256) of a u64 and a u32;
+// named barrier 1 over those 256 threads.
+__device__ __forceinline__ void digit_scan2(uint64_t m, uint32_t c, uint64_t* wm, uint32_t* wc, uint64_t& sm,
+                                            uint32_t& sc) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint64_t xm = m;
+  uint32_t xc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t ym = __shfl_up_sync(0xffffffffu, xm, o);
+    const uint32_t yc = __shfl_up_sync(0xffffffffu, xc, o);
+    if (lane >= o) {
+      xm += ym;
+      xc += yc;
+    }
+  }
+  if (lane == 31) {
+    wm[wid] = xm;
+    wc[wid] = xc;
+  }
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+  uint64_t om = 0u;
+  uint32_t oc = 0u;
+  for (int w = 0; w < wid; ++w) {
+    om += wm[w];
+    oc += wc[w];
+  }
+  sm = om + xm;
+  sc = oc + xc;
+}
 
 // Exclusive block scan of one u32 per thread (all kThreads threads call it).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t& total) {
@@ -71,7 +127,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   const int g = blockIdx.y, b = blockIdx.z;
   const int grp = b * a.Hkv + g;
   const int L = a.L;
-  const int K = a.kept.kept[grp];
+  int K = a.kept.kept[grp];
   const float* sc = a.scores + (size_t)grp * L;
   int32_t* pm = a.perm + (size_t)grp * L;
   const int per = (L + kClusterCtas - 1) / kClusterCtas;
@@ -84,10 +140,92 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   __shared__ uint32_t dig_warp[8];
   __shared__ uint32_t sh_digit, sh_above;
   __shared__ uint32_t cnt[2];  // this slice's (#key > T, #key == T)
+  __shared__ uint64_t histm[2][256];  // coverage mode: mass per digit
+  __shared__ uint64_t dig_warp_m[8];
+  __shared__ uint64_t sh_mass, sh_mabove;
+
+  uint32_t prefix = 0u, mask = 0u, krem = 0u;
+  bool have_T = false;  // coverage mode found the K-th key by mass
+  if (a.coverage) {
+    if (tid == 0) sh_mass = 0u;
+    __syncthreads();
+    uint64_t my = 0u;
+    for (int i = lo + tid; i < hi; i += kThreads) my += token_mass(sc[i], a.mass_scale);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) my += __shfl_xor_sync(0xffffffffu, my, o);
+    if ((tid & 31) == 0 && my) atomicAdd(reinterpret_cast<unsigned long long*>(&sh_mass), (unsigned long long)my);
+    cluster.sync();
+    uint64_t M = 0u;
+    for (int r = 0; r < kClusterCtas; ++r) M += *cluster.map_shared_rank(&sh_mass, r);
+    const uint64_t D = (uint64_t)floor(__ull2double_rn(M) * a.tau);
+    uint64_t trem = D >= M ? 0u : M - D;
+    if (trem == 0u) {
+      K = 1;  // nothing has to be covered: keep the single top token
+    } else {
+      uint32_t above = 0u;
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        uint32_t* hc = hist[pass & 1];
+        uint64_t* hm = histm[pass & 1];
+        if (tid < 256) {
+          hc[tid] = 0u;
+          hm[tid] = 0u;
+        }
+        __syncthreads();
+        for (int i = lo + tid; i < hi; i += kThreads) {
+          const float f = sc[i];
+          const uint32_t key = order_key(f);
+          if ((key & mask) == prefix) {
+            const uint32_t dg = (key >> shift) & 255u;
+            atomicAdd(&hc[dg], 1u);
+            const uint64_t m = token_mass(f, a.mass_scale);
+            if (m) atomicAdd(reinterpret_cast<unsigned long long*>(&hm[dg]), (unsigned long long)m);
+          }
+        }
+        cluster.sync();
+        if (tid < 256) {
+          // Thread t stands for digit 255 - t: inclusive scans give the count
+          // and mass of matching keys whose digit is >= 255 - t.
+          uint32_t totc = 0u;
+          uint64_t totm = 0u;
+          for (int r = 0; r < kClusterCtas; ++r) {
+            totc += cluster.map_shared_rank(hc, r)[255 - tid];
+            totm += cluster.map_shared_rank(hm, r)[255 - tid];
+          }
+          uint64_t Sm;
+          uint32_t Sc;
+          digit_scan2(totm, totc, dig_warp_m, dig_warp, Sm, Sc);
+          if (Sm >= trem && Sm - totm < trem) {
+            sh_digit = 255u - (uint32_t)tid;
+            sh_mabove = Sm - totm;
+            sh_above = Sc - totc;
+          }
+        }
+        __syncthreads();
+        prefix |= sh_digit << shift;
+        mask |= 0xFFu << shift;
+        trem -= sh_mabove;
+        above += sh_above;
+      }
+      // Every key equal to the K-th carries the same mass, which is > 0
+      // because that key's digit raised the running mass to the target.
+      const uint64_t mk = token_mass(key_to_float(prefix), a.mass_scale);
+      uint64_t need = 1u;
+      if (mk == 0u) {
+        record_status(a.status, TSA_ERR_DEVICE_BOUNDS);
+      } else {
+        need = (trem + mk - 1u) / mk;
+      }
+      K = (int)min((uint64_t)L, (uint64_t)above + need);
+      krem = (uint32_t)K - above;
+      have_T = true;
+    }
+    if (a.k_out && rank == 0 && tid == 0) a.k_out[grp] = K;
+  }
 
   const bool partial = K < L;
-  uint32_t prefix = 0u, mask = 0u, krem = (uint32_t)K;
-  if (partial) {
+  if (!have_T) krem = (uint32_t)K;
+  if (partial && !have_T) {
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       uint32_t* h = hist[pass & 1];
@@ -210,7 +348,32 @@ cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kep
   a.status = status;
   a.L = d.L;
   a.Hkv = d.Hkv;
+  a.coverage = 0;
+  a.tau = 0.0;
+  a.mass_scale = 0.f;
+  a.k_out = nullptr;
   a.kept = kept;
+  const dim3 grid(kClusterCtas, d.Hkv, d.B);
+  select_radix<<<grid, kThreads, 0, st>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_coverage(const Dims& d, const float* scores, double tau, int32_t* perm, int32_t* k_out,
+                                   uint32_t* status, cudaStream_t st) {
+  SelectArgs a;
+  a.scores = scores;
+  a.perm = perm;
+  a.status = status;
+  a.L = d.L;
+  a.Hkv = d.Hkv;
+  a.coverage = 1;
+  a.tau = tau;
+  int lg = 0;  // ceil(log2 L)
+  while ((1ll << lg) < (long long)d.L) ++lg;
+  a.mass_scale = ldexpf(1.f, 55 - lg);
+  a.k_out = k_out;
+  for (int i = 0; i < kMaxGroups; ++i) a.kept.kept[i] = 0;
   const dim3 grid(kClusterCtas, d.Hkv, d.B);
   select_radix<<<grid, kThreads, 0, st>>>(a);
   count_launches(1);

@@ -54,6 +54,8 @@ WsLayout ws_layout(const Dims& d, int window) {
   off += align256((size_t)d.B * d.Hkv * kMaxScoreSplits * Mp * 2 * sizeof(float));
   w.lse = off;
   off += align256((size_t)d.B * d.Hkv * Mp * sizeof(float));
+  w.budgets = off;
+  off += align256((size_t)kMaxGroups * sizeof(int32_t));
   w.total = off;
   return w;
 }
@@ -188,6 +190,20 @@ tsa_status tsa_select(const tsa_desc* desc, const float* scores, const int32_t* 
   return run_select(d, scores, kb, perm, ws, static_cast<cudaStream_t>(stream));
 }
 
+tsa_status tsa_select_coverage(const tsa_desc* desc, const float* scores, double tau, int32_t* perm,
+                               int32_t* budget_dev_out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!(tau >= 0.0 && tau <= 1.0)) return TSA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!aligned16(scores) || !aligned16(perm) || !aligned16(ws) || budget_dev_out == nullptr ||
+      (reinterpret_cast<uintptr_t>(budget_dev_out) & 3u) != 0)
+    return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  return cuda_status(launch_select_coverage(d, scores, tau, perm, budget_dev_out, status_word(ws),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const void* v, const int32_t* perm,
                       const int32_t* budget_host, void* out, void* ws, size_t ws_bytes, void* stream) {
   Dims d;
@@ -261,6 +277,35 @@ tsa_status tsa_forward(const tsa_desc* desc, const void* q, const void* k, const
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = run_score(d, q, k, window, scores, ws, st)) != TSA_OK) return s;
   if ((s = run_select(d, scores, kb, perm, ws, st)) != TSA_OK) return s;
+  return run_attend(d, q, k, v, perm, kb, out, ws, st);
+}
+
+tsa_status tsa_forward_coverage(const tsa_desc* desc, const void* q, const void* k, const void* v, int32_t window,
+                                double tau, int32_t* budget_host_out, float* scores_or_null, int32_t* perm_or_null,
+                                void* out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if ((s = check_window(d, window)) != TSA_OK) return s;
+  if (!(tau >= 0.0 && tau <= 1.0) || budget_host_out == nullptr) return TSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+    return TSA_ERR_INVALID_ARG;
+  if ((scores_or_null && !aligned16(scores_or_null)) || (perm_or_null && !aligned16(perm_or_null)))
+    return TSA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(d, window);
+  if (ws_bytes < w.total) return TSA_ERR_WORKSPACE;
+  float* scores = scores_or_null ? scores_or_null : ws_ptr<float>(ws, w.scores);
+  int32_t* perm = perm_or_null ? perm_or_null : ws_ptr<int32_t>(ws, w.perm);
+  int32_t* kdev = ws_ptr<int32_t>(ws, w.budgets);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = run_score(d, q, k, window, scores, ws, st)) != TSA_OK) return s;
+  if ((s = cuda_status(launch_select_coverage(d, scores, tau, perm, kdev, status_word(ws), st))) != TSA_OK) return s;
+  // The attention grid is sized from the budgets, so they come back to the host here.
+  const size_t nb = (size_t)d.B * d.Hkv * sizeof(int32_t);
+  if ((s = cuda_status(cudaMemcpyAsync(budget_host_out, kdev, nb, cudaMemcpyDeviceToHost, st))) != TSA_OK) return s;
+  if ((s = cuda_status(cudaStreamSynchronize(st))) != TSA_OK) return s;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host_out, &kb)) != TSA_OK) return s;
   return run_attend(d, q, k, v, perm, kb, out, ws, st);
 }
 

@@ -133,7 +133,10 @@ def make_scores(B: int, Hkv: int, L: int, seed: int = 0, kind: str = "random") -
           "ties"    values from a small set, so many ties sit at any threshold;
           "equal"   all equal;
           "zeros"   mix of +0.0 and -0.0 with a few positive values;
-          "denorm"  subnormal and tiny normal values.
+          "denorm"  subnormal and tiny normal values;
+          "peaked"  log-normal exp(3 N(0,1)) values scaled to sum to 256 per
+                    head, like window scores (G * W = 256 probability rows)
+                    concentrated on a few keys.
     """
     g = torch.Generator(device="cpu").manual_seed(seed)
     if kind == "random":
@@ -152,6 +155,9 @@ def make_scores(B: int, Hkv: int, L: int, seed: int = 0, kind: str = "random") -
     if kind == "denorm":
         e = torch.randint(-149, -120, (B, Hkv, L), generator=g).float()
         return torch.pow(2.0, e)
+    if kind == "peaked":
+        x = torch.exp(3.0 * torch.randn((B, Hkv, L), generator=g, dtype=torch.float64))
+        return (256.0 * x / x.sum(-1, keepdim=True)).float()
     raise ValueError(kind)
 
 
