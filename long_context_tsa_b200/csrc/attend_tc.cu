@@ -1,5 +1,6 @@
 // Compressed causal attention on the tcgen05 tensor cores (bf16 in, fp32
-// accumulate), with the gather fused into TMA tile::gather4 loads and the
+// accumulate), with the gather fused into the loads (16-byte cp.async copies of
+// the selected rows straight into the swizzled shared-memory tiles) and the
 // scatter fused into the epilogue.
 //
 // "Token Sparse Attention Long Context" (skill page), Steps 2-3;
@@ -36,6 +37,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "device_common.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
@@ -55,7 +58,6 @@ constexpr int kZeroWarps = 3;
 constexpr uint32_t kTeardownPolls = 1u << 26;
 constexpr long long kFusedZeroMinCtas = 2 * 148;  // attention CTAs from which the zero fill is fused
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr float kRescaleBound = 256.0f;     // 2^kRescaleThreshold: the largest P kept without a rescale
 
 struct TcAttendParams {
   const __nv_bfloat16* q;
@@ -339,94 +341,51 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     const int pos = c * P2 + t * p.RP + (r - hh * p.RP);
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    // The two softmax warpgroups take turns (named barriers 1 and 2): at d = 128
-    // the exponentials of one tile keep MUFU as busy as the MMAs of the other
-    // tile keep the tensor core, so the tiles alternate instead of sharing MUFU.
-    // Every iteration performs its barrier operations whatever happens (also
-    // after a timeout), and the arrive counts match the syncs exactly: tile 0
-    // goes first; tile 1 skips its last arrive.
-    const uint32_t bar_mine = 1u + (uint32_t)t, bar_other = 2u - (uint32_t)t;
-    if (t == 1) named_arrive(1u, 256u);
+    // The two softmax warpgroups run independently: while one is in its
+    // latency-bound max pass the other keeps the exponential unit busy.  (Taking
+    // strict turns on the whole softmax phase measured 8 % slower.)
     for (int j = 0; j < n_kt; ++j) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
-      named_sync(bar_mine, 256u);
-      if (!ok) {
-        if (!(t == 1 && j == n_kt - 1)) named_arrive(bar_other, 256u);
-        continue;
-      }
+      if (!ok) continue;
       tc_fence_after();
       const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
       // Only tiles on the diagonal hide keys from some rows (warp-uniform choice).
       const bool masked = __any_sync(0xffffffffu, nvis < 128);
-      // Fast path (tiles after the first): one pass per 32-column chunk against the
-      // current reference max m, t = x * scale - m, P = 2^t written to TMEM at
-      // once (bf16 pairs over S columns [16 q, 16 q + 16), which were already
-      // read).  A chunk where some row has t > threshold (warp vote) switches the
-      // warp to the exact path: the new reference is that row's exact max over the
-      // unread chunks (the written ones had t <= threshold), the written P chunks
-      // are rescaled in TMEM by alpha = 2^(m - m_new) <= 2^-threshold, and the rest
-      // of the row is computed against m_new.  The first tile always takes the
-      // exact two-pass path.
-      const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-      uint64_t acc2 = 0ull;  // packed fp32 pair of the running row sum
-      auto xval = [&](const uint32_t* v, int q4, int e) -> float {
-        const float x = __uint_as_float(v[e]);
-        return (!masked || q4 * 32 + e < nvis) ? x : -INFINITY;
-      };
+      // Two passes over S_t, each in four 32-column chunks whose TMEM loads run one
+      // chunk ahead (registers va / vb alternate).  Pass 1: the row max x_max.  The
+      // reference m moves only when x_max * scale exceeds it by more than the
+      // threshold (always on the first tile, where m = -inf); then alpha =
+      // 2^(m_old - m_new) rescales l and O.  Pass 2: P = 2^(x * scale - m) for every
+      // column against that final m (so P <= 2^threshold), summed into l and written
+      // to TMEM as bf16 pairs over S columns [16 q, 16 q + 16), which pass 2 has
+      // already read.  No decision inside the exponential loop.
       float alpha = 1.f;
       bool rescaled = false;  // warp-uniform: O must be rescaled by alpha
-      int q_bad = 4;          // first chunk with a violation (4 = none)
-      if (j > 0) {
-        const uint64_t negm2 = f2_pack(-m_use, -m_use);
-        // S chunks are double-buffered in registers: the load of chunk q + 1 is in
-        // flight while chunk q is processed.
+      uint64_t acc2 = 0ull;   // packed fp32 pair of the tile's row sum
+      auto tile = [&](auto masked_c) {
+        constexpr bool kMasked = decltype(masked_c)::value;
+        auto xval = [&](const uint32_t* v, int q4, int e) -> float {
+          const float x = __uint_as_float(v[e]);
+          return (!kMasked || q4 * 32 + e < nvis) ? x : -INFINITY;
+        };
         uint32_t va[32], vb[32];
         tmem_ld32(tS, va);
+        float mxs[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t(&v)[32] = (q4 & 1) ? vb : va;
           uint32_t(&vn)[32] = (q4 & 1) ? va : vb;
-          if (q4 < 3) tmem_ld32_async(tS + (q4 + 1) * 32, vn);
-          // P of this chunk in registers; its largest value decides (P > 2^threshold
-          // <=> t > threshold) before anything is written.
-          uint32_t pk[16];
-          uint64_t accq[2] = {0ull, 0ull};
-          __nv_bfloat162 pm2[2] = {__floats2bfloat162_rn(0.f, 0.f), __floats2bfloat162_rn(0.f, 0.f)};
+          tmem_ld32_async(tS + ((q4 + 1) & 3) * 32, vn);  // after chunk 3: pass 2's chunk 0
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            float t0, t1;
-            f2_unpack(f2_fma(f2_pack(xval(v, q4, 2 * e2), xval(v, q4, 2 * e2 + 1)), scale2, negm2), t0, t1);
-            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-            accq[e2 & 1] = f2_add(accq[e2 & 1], f2_pack(p0, p1));
-            pk[e2] = pack_bf16(p0, p1);
-            pm2[e2 & 1] = __hmax2(pm2[e2 & 1], *reinterpret_cast<const __nv_bfloat162*>(&pk[e2]));
+          for (int e = 0; e < 32; e += 8) {
+            mxs[0] = fmax3(mxs[0], xval(v, q4, e), xval(v, q4, e + 1));
+            mxs[1] = fmax3(mxs[1], xval(v, q4, e + 2), xval(v, q4, e + 3));
+            mxs[2] = fmax3(mxs[2], xval(v, q4, e + 4), xval(v, q4, e + 5));
+            mxs[3] = fmax3(mxs[3], xval(v, q4, e + 6), xval(v, q4, e + 7));
           }
-          const __nv_bfloat162 pmx = __hmax2(pm2[0], pm2[1]);
-          const float pmax = fmaxf(__bfloat162float(pmx.x), __bfloat162float(pmx.y));
-          const bool bad = __any_sync(0xffffffffu, pmax > kRescaleBound);
-          if (q4 < 3) tmem_wait_ld32(vn);  // no load left in flight, whatever happens next
-          if (bad) {
-            q_bad = q4;
-            break;
-          }
-          tmem_st16(tS + q4 * 16, pk);
-          acc2 = f2_add(acc2, f2_add(accq[0], accq[1]));
+          tmem_wait_ld32(vn);
         }
-      } else {
-        q_bad = 0;
-      }
-      if (q_bad < 4) {
-        // Exact path from chunk q_bad on.  New reference: the exact max of the
-        // unread chunks for rows that exceed the threshold (or every row on the
-        // first tile, where m is -inf).
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int q4 = q_bad; q4 < 4; ++q4) {
-          uint32_t v[32];
-          tmem_ld32(tS + q4 * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, xval(v, q4, e));
-        }
+        const float mx = fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3]));
         const float mt = mx * p.scale_log2;
         const bool need = mt > m_use + kRescaleThreshold;  // always true on the first tile
         if (need) {
@@ -434,40 +393,37 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           m_use = mt;
         }
         rescaled = j > 0 && __any_sync(0xffffffffu, need);
-        // Written chunks: P *= alpha (they were computed against the old reference).
-        if (rescaled) {
-          float a0, a1;
-          f2_unpack(acc2, a0, a1);
-          acc2 = f2_pack(a0 * alpha, a1 * alpha);
-#pragma unroll 1
-          for (int q4 = 0; q4 < q_bad; ++q4) {
-            uint32_t w[32];
-            tmem_ld32(tS + q4 * 16, w);  // 32 columns: chunks q4 and q4 + 1 of P (16 used)
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-              pk[e] = pack_bf16(__bfloat162float(h.x) * alpha, __bfloat162float(h.y) * alpha);
-            }
-            tmem_st16(tS + q4 * 16, pk);
-          }
-        }
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
+        uint64_t accq[2] = {0ull, 0ull};
+        // Pairs of chunks per iteration of a rolled loop: the loop edge keeps the
+        // scheduler from interleaving all four chunks (which ran out of registers).
 #pragma unroll 1
-        for (int q4 = q_bad; q4 < 4; ++q4) {
-          uint32_t v[32];
-          tmem_ld32(tS + q4 * 32, v);
+        for (int qq = 0; qq < 4; qq += 2)
+#pragma unroll
+        for (int qi = 0; qi < 2; ++qi) {
+          const int q4 = qq + qi;
+          uint32_t(&v)[32] = qi ? vb : va;  // pass 2's chunk 0 sits in va
+          uint32_t(&vn)[32] = qi ? va : vb;
+          if (q4 < 3) tmem_ld32_async(tS + (q4 + 1) * 32, vn);
           uint32_t pk[16];
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
             float t0, t1;
             f2_unpack(f2_fma(f2_pack(xval(v, q4, 2 * e2), xval(v, q4, 2 * e2 + 1)), scale2, negm2), t0, t1);
             const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-            acc2 = f2_add(acc2, f2_pack(p0, p1));
+            accq[e2 & 1] = f2_add(accq[e2 & 1], f2_pack(p0, p1));
             pk[e2] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + q4 * 16, pk);
+          if (q4 < 3) tmem_wait_ld32(vn);
         }
+        acc2 = f2_add(accq[0], accq[1]);
+      };
+      if (masked) {
+        tile(std::true_type{});
+      } else {
+        tile(std::false_type{});
       }
       {
         float s0, s1;
@@ -490,7 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       tmem_st_wait();  // P (and a rescaled O) are in TMEM before the MMA warp is told
       tc_fence_before();
       mbar_arrive(bar_p(t));
-      if (!(t == 1 && j == n_kt - 1)) named_arrive(bar_other, 256u);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o(t), 0, p.wait_limit, abort_flag));
     if (!ok) {
