@@ -30,6 +30,10 @@ What it computes (each function cites the passage it follows):
   score, made exact by fixed point -- floor(clamp(s, 0, 256) * 2^S) as an
   integer, S = 55 - ceil(log2 L) so that a head's total stays below 2^63 --
   and the dropped mass may be at most floor(double(M) * tau) of the total M.
+* ``attend_block_sparse`` -- ``attend`` restricted further by a mask over
+  128 x 128 blocks of the compressed (query, key) space.  Source: the
+  sciencestack page, Figures 1 and 5b (Token Sparse Attention composed with a
+  block-sparse attention kernel inside the compressed token set).
 * ``drift``   -- representation drift between two hidden-state tensors:
   one minus the mean, over all (batch, position) rows, of the cosine of the
   two rows after each is divided by max(its L2 norm, eps).  Source: the skill
@@ -73,6 +77,8 @@ __all__ = [
     "attend",
     "attend_rows",
     "attend_accumulate",
+    "attend_block_sparse",
+    "BLOCK",
     "forward",
     "row_cosine",
     "drift",
@@ -216,7 +222,8 @@ def coverage_budgets(scores, tau: float) -> np.ndarray:
     return out
 
 
-def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=None) -> np.ndarray:
+def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=None,
+                block_mask_bg=None) -> np.ndarray:
     """Output rows for query head h of batch b at compacted indices ``rows``.
 
     Compacted row i stands for original position p_i = perm_bg[i] (i < K).
@@ -224,6 +231,11 @@ def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=No
     kept rows r whose original position p_r <= p_i (causal by original
     positions).  Returns [len(rows), D] float64.  This is Step 3's
     matmul / softmax / matmul on the gathered tensors of Step 2.
+
+    ``block_mask_bg`` (optional, [nb, nb] of bool, nb >= ceil(K / BLOCK)) adds
+    the block-sparse composition: key r is visible to row i only when
+    block_mask_bg[i // BLOCK, r // BLOCK] is set as well.  A row that sees no
+    key at all outputs zeros.
     """
     D = np.shape(q)[-1]
     s = _scale(D, scale)
@@ -239,11 +251,51 @@ def attend_rows(q, k, v, perm_bg, K: int, b: int, h: int, G: int, rows, scale=No
         pq = idx[rr]  # original positions of these queries
         qh = _f64(q[b, h][pq])  # [n, D]  gathered queries
         logits = s * (qh @ kh.T)  # [n, K]
-        logits = np.where(idx[None, :] <= pq[:, None], logits, -np.inf)
+        visible = idx[None, :] <= pq[:, None]
+        if block_mask_bg is not None:
+            bm = np.asarray(block_mask_bg, dtype=bool)
+            visible = visible & bm[(rr // BLOCK)[:, None], (np.arange(K) // BLOCK)[None, :]]
+        logits = np.where(visible, logits, -np.inf)
         m = logits.max(axis=1, keepdims=True)
+        empty = ~np.isfinite(m[:, 0])
+        m = np.where(np.isfinite(m), m, 0.0)
         e = np.exp(logits - m)
-        p = e / e.sum(axis=1, keepdims=True)
+        den = e.sum(axis=1, keepdims=True)
+        p = e / np.where(empty[:, None], 1.0, den)
         out[c0:c0 + chunk] = p @ vh
+    return out
+
+
+# Block size (in compacted positions and keys) of the block-sparse composition.
+BLOCK = 128
+
+
+def attend_block_sparse(q, k, v, perm, budgets, block_mask, scale=None) -> np.ndarray:
+    """``attend`` composed with a block mask over the compressed space.
+
+    ``block_mask`` is [B, Hkv, nb, nb] (nb = ceil(L / BLOCK)), nonzero where
+    the block of compacted query rows [BLOCK * i, BLOCK * i + BLOCK) may attend
+    to the block of compacted keys [BLOCK * j, ...); the causal mask still
+    applies inside.  Source: "Token Sparse Attention: Efficient Long-Context
+    Inference with Interleaved Token Selection" (sciencestack), Figures 1 and
+    5b (the method applied on top of a block-sparse attention kernel inside
+    the compressed token set).  Reading: the mask is given per KV group in
+    compacted coordinates; rows that see no key output zeros; dropped rows are
+    zeros as in ``attend``.
+    """
+    B, Hq, L, D = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    kept = clamp_budgets(budgets, L)
+    perm = np.asarray(perm, dtype=np.int64)
+    bm = np.asarray(block_mask) != 0
+    out = np.zeros((B, Hq, L, D), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            K = int(kept[b * Hkv + g])
+            out[b, h, perm[b, g, :K]] = attend_rows(q, k, v, perm[b, g], K, b, h, G, np.arange(K), scale,
+                                                    block_mask_bg=bm[b, g])
     return out
 
 

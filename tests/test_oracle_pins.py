@@ -461,3 +461,64 @@ def test_coverage_minimality_and_monotonicity():
             if K > 1:  # ... and the best K - 1 do not
                 best = np.sort(m)[::-1][:K - 1]
                 assert int(best.sum()) < T
+
+
+# --- block-sparse composition --------------------------------------------------------------
+
+
+def _block_full_mask(perm_bg, K, L, bm):
+    """Full-length boolean mask M[p, p'] of block-sparse attention in the compressed
+    space, written out in original coordinates from first principles."""
+    M = np.zeros((L, L), dtype=bool)
+    pos = perm_bg[:K]
+    for i in range(K):
+        for r in range(i + 1):  # causal on compacted indices
+            if bm[i // 128, r // 128]:
+                M[pos[i], pos[r]] = True
+    return M
+
+
+def test_block_sparse_matches_sdpa_with_explicit_mask():
+    B, Hq, Hkv, L, D = 1, 2, 1, 700, 8
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    budgets = [600]
+    perm = O.select(rng.random((B, Hkv, L)), budgets)
+    nb = -(-L // 128)
+    bm = rng.random((B, Hkv, nb, nb)) < 0.5
+    bm[0, 0, 2, 2] = False  # a diagonal block off: its early rows see only earlier blocks
+    bm[0, 0, 0, 0] = False  # block 0 sees nothing at all: its rows are zeros
+    out = O.attend_block_sparse(q, k, v, perm, budgets, bm)
+    M = _block_full_mask(perm[0, 0], 600, L, bm[0, 0])
+    rows = M.any(axis=1)
+    ref = _sdpa64(q, k, v, mask=M)
+    np.testing.assert_allclose(out[0][:, rows], ref[0][:, rows], rtol=0, atol=1e-12)
+    kept = np.zeros(L, bool)
+    kept[perm[0, 0, :600]] = True
+    assert np.all(out[0][:, ~rows] == 0.0)  # no visible key, or dropped
+    assert np.all(out[0][:, perm[0, 0, :128]] == 0.0)  # the rows of block 0
+
+
+def test_block_sparse_full_mask_is_attend_and_diagonal_mask_is_blockwise():
+    B, Hq, Hkv, L, D = 1, 4, 2, 520, 8
+    q = rng.standard_normal((B, Hq, L, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    budgets = [400, 520]
+    perm = O.select(rng.random((B, Hkv, L)), budgets)
+    nb = -(-L // 128)
+    full = np.ones((B, Hkv, nb, nb), dtype=np.uint8)
+    np.testing.assert_array_equal(O.attend_block_sparse(q, k, v, perm, budgets, full),
+                                  O.attend(q, k, v, perm, budgets))
+    diag = np.broadcast_to(np.eye(nb, dtype=np.uint8), (B, Hkv, nb, nb))
+    out = O.attend_block_sparse(q, k, v, perm, budgets, diag)
+    for g, K in enumerate(budgets):
+        for blk in range(0, K, 128):
+            sub = perm[:, g:g + 1, blk:min(K, blk + 128)]  # the block as its own sequence
+            n = sub.shape[-1]
+            sub_perm = np.broadcast_to(np.arange(n), (1, 1, n))
+            hs = slice(2 * g, 2 * g + 2)
+            ref = O.attend(q[:, hs][:, :, sub[0, 0]], k[:, g:g + 1][:, :, sub[0, 0]], v[:, g:g + 1][:, :, sub[0, 0]],
+                           sub_perm, [n])
+            np.testing.assert_allclose(out[0, hs][:, sub[0, 0]], ref[0], rtol=0, atol=1e-12)
