@@ -57,6 +57,33 @@ def attend_flops(w, budgets) -> float:
     return total
 
 
+def block_mask_for(w, density: float, seed: int = 5) -> np.ndarray:
+    """Seeded uint8 [B, Hkv, nb, nb] block mask: diagonal blocks, the first block column
+    (attention sinks) and a `density` fraction of the other blocks."""
+    nb = -(-w.L // 128)
+    rng = np.random.default_rng(seed)
+    bm = (rng.random((w.B, w.Hkv, nb, nb)) < density).astype(np.uint8)
+    bm[:, :, np.arange(nb), np.arange(nb)] = 1
+    bm[:, :, :, 0] = 1
+    return bm
+
+
+def block_sparse_flops(w, budgets, bm) -> float:
+    """Flops of the visible (query, key) pairs: causal inside enabled 128 x 128 blocks."""
+    total = 0.0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            K = min(budgets[b * w.Hkv + g], w.L)
+            n = -(-K // 128)
+            sizes = np.minimum(128, K - 128 * np.arange(n)).astype(np.float64)
+            m = bm[b, g, :n, :n].astype(bool)
+            low = np.tril(m, -1)
+            pairs = (sizes[:, None] * sizes[None, :] * low).sum()
+            pairs += (sizes * (sizes + 1) / 2 * np.diag(m)).sum()
+            total += w.G * 4.0 * w.D * pairs
+    return total
+
+
 def rank_seed(rank: int) -> int:
     """Each rank runs its own independent layer (weak scaling): inputs seeded by rank."""
     return rank
@@ -234,11 +261,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="forward", choices=["forward", "forward-accumulate", "forward-coverage", "drift"],
+    ap.add_argument("--op", default="forward",
+                    choices=["forward", "forward-accumulate", "forward-coverage", "forward-block-sparse", "drift"],
                     help="forward: score/select/attend (the headline); forward-accumulate: the same with the "
                          "scatter-add attention into a resident output; forward-coverage: budgets chosen per KV "
-                         "head from the coverage --tau (one device-to-host copy of the budgets per step); drift: "
-                         "the representation-drift pass")
+                         "head from the coverage --tau (one device-to-host copy of the budgets per step); "
+                         "forward-block-sparse: attention restricted by a 128 x 128 block mask of --density in the "
+                         "compressed space; drift: the representation-drift pass")
+    ap.add_argument("--density", type=float, default=0.5, help="block density for --op forward-block-sparse")
     ap.add_argument("--tau", type=float, default=0.005, help="token coverage for --op forward-coverage")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -280,6 +310,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
     accumulate = args.op == "forward-accumulate"
     coverage = args.op == "forward-coverage"
+    block_sparse = args.op == "forward-block-sparse"
+    bm_host = block_mask_for(w, args.density) if block_sparse else None
+    bm_dev = torch.from_numpy(bm_host).to(dev) if block_sparse else None
     if accumulate:
         out.normal_()  # the residual the attention output is added into
     kdev = torch.empty(w.B * w.Hkv, dtype=torch.int32, device=dev)
@@ -300,6 +333,8 @@ def main():
             ev[2].record(stream)
         if accumulate:
             T.tsa_attend_accumulate(desc, q, k, v, perm, budgets, out, ws)
+        elif block_sparse:
+            T.tsa_attend_block_sparse(desc, q, k, v, perm, budgets, bm_dev, out, ws)
         else:
             T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
         if ev is not None:
@@ -345,7 +380,7 @@ def main():
     value = job_tokens_per_s(world, tokens, ms_per_step)
 
     peaks, peak_src = load_peaks()
-    flops = attend_flops(w, budgets)
+    flops = block_sparse_flops(w, budgets, bm_host) if block_sparse else attend_flops(w, budgets)
     achieved = flops / (t_attend / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
@@ -381,6 +416,7 @@ def main():
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "op": args.op, "tau": args.tau if args.op == "forward-coverage" else None,
+                   "block_density": args.density if block_sparse else None,
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets,
                    "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "

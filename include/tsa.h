@@ -144,6 +144,24 @@ TSA_API tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const 
                                      float* scores, void* stream);
 
 /*
+ * tsa_attend_block_sparse -- tsa_attend composed with block-sparse attention
+ * inside the compressed space ("Token Sparse Attention: Efficient Long-Context
+ * Inference with Interleaved Token Selection", Figures 1 and 5b: the method on
+ * top of a block-sparse attention kernel).  block_mask: device uint8
+ * [B*Hkv][nb][nb], nb = ceil(L / 128), row-major; entry (i, j) of KV group
+ * (b, g) enables the block of compacted query rows [128 i, 128 i + 128) of its
+ * G query heads against compacted keys [128 j, 128 j + 128); the causal mask
+ * still applies inside.  Disabled key tiles are skipped (no loads, no MMAs)
+ * when every query row of a CTA has them disabled.  A kept row that sees no
+ * key outputs zeros; dropped rows are zeros as in tsa_attend.  Same other
+ * arguments and rules as tsa_attend.
+ */
+TSA_API tsa_status tsa_attend_block_sparse(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                                           const int32_t* perm, const int32_t* budget_host,
+                                           const uint8_t* block_mask, void* out, void* ws, size_t ws_bytes,
+                                           void* stream);
+
+/*
  * tsa_select_coverage -- tsa_select with each (b, g) budget chosen from a
  * token coverage tau in [0, 1] ("Token Sparse Attention: Efficient
  * Long-Context Inference with Interleaved Token Selection": dynamic token

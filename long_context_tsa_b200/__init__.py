@@ -17,6 +17,7 @@ from ._native import (  # noqa: F401
     make_desc,
     tsa_attend,
     tsa_attend_accumulate,
+    tsa_attend_block_sparse,
     tsa_check_status,
     tsa_debug_launch_count,
     tsa_debug_set_wait_limit,

@@ -24,7 +24,7 @@ EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
-            "tsa_select_coverage", "tsa_forward_coverage")
+            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse")
 
 
 class TsaDesc(ctypes.Structure):
@@ -59,6 +59,7 @@ _SIGS = {
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_attend_block_sparse": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_select_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, ctypes.c_double, _P, _P, _P, _SZ, _P]),
     "tsa_forward_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P,
                                             _P, _P, _SZ, _P]),
@@ -241,3 +242,15 @@ def tsa_forward_coverage(desc, q, k, v, window, tau, out, ws, scores=None, perm=
                                       _ptr(scores), _ptr(perm), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "tsa_forward_coverage")
     return list(arr)
+
+
+def tsa_attend_block_sparse(desc, q, k, v, perm, budgets, block_mask, out, ws, stream=None):
+    """tsa_attend restricted by a uint8 [B, Hkv, nb, nb] mask over 128 x 128 blocks of compacted (query, key)."""
+    nb = (desc.L + 127) // 128
+    if block_mask.dtype != torch.uint8 or block_mask.numel() != desc.B * desc.Hkv * nb * nb:
+        raise ValueError("block_mask must be uint8 [B, Hkv, ceil(L/128), ceil(L/128)]")
+    if not block_mask.is_contiguous():
+        raise ValueError("block_mask must be contiguous")
+    _check(lib().tsa_attend_block_sparse(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
+                                         _ptr(block_mask), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "tsa_attend_block_sparse")

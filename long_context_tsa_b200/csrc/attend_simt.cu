@@ -32,6 +32,8 @@ struct AttendArgs {
   int Hq, Hkv, L, G;
   float scale;
   int accumulate;  // 1: out[kept rows] += attention
+  const uint8_t* bmask;  // [B*Hkv][nb][nb] block mask over compacted (query, key) 128-blocks, or null
+  int nb;
   Budgets kept;
 };
 
@@ -96,7 +98,9 @@ __global__ void __launch_bounds__(256) attend_simt(AttendArgs a) {
   }
 
   const int nkeys = min(K, r0 + BR);
+  const uint8_t* bm = a.bmask ? a.bmask + ((size_t)grp * a.nb + r0 / 128) * a.nb : nullptr;  // this CTA's block row
   for (int c0 = 0; c0 < nkeys; c0 += BC) {
+    if (bm != nullptr && bm[c0 / 128] == 0) continue;  // block disabled (uniform over the CTA)
     __syncthreads();
     for (int idx = tid; idx < BC * D; idx += blockDim.x) {
       const int n = idx / D, d = idx - n * D;
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(256) attend_simt(AttendArgs a) {
     const int r = r0 + ty * 4 + i;
     if (r < K) {
       const size_t p = (size_t)checked_pos(pm, r, L, a.status);
-      const float inv = 1.f / l_i[i];
+      const float inv = l_i[i] > 0.f ? 1.f / l_i[i] : 0.f;  // no visible key (block mask): zeros
 #pragma unroll
       for (int dc = 0; dc < DC; ++dc) {
         T* dst = oh + p * D + tx + 16 * dc;
@@ -234,6 +238,8 @@ AttendArgs make_args(const Dims& d, const void* q, const void* k, const void* v,
   a.G = d.G;
   a.scale = d.scale;
   a.accumulate = 0;
+  a.bmask = nullptr;
+  a.nb = (d.L + 127) / 128;
   a.kept = kept;
   return a;
 }
@@ -272,9 +278,10 @@ void kept_range(const Dims& d, const Budgets& kept, int& mn, int& mx) {
 
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
-                               bool accumulate, cudaStream_t st) {
+                               bool accumulate, const uint8_t* block_mask, cudaStream_t st) {
   AttendArgs a = make_args(d, q, k, v, perm, kept, out, status);
   a.accumulate = accumulate ? 1 : 0;
+  a.bmask = block_mask;
   int mn, mx;
   kept_range(d, kept, mn, mx);
   if (d.dtype == TSA_F32)

@@ -71,6 +71,8 @@ struct TcAttendParams {
   uint64_t wait_limit;
   int accumulate;  // 1: out[kept rows] += attention, dropped rows untouched
   int zero_fill;   // 1: warps 13-15 write the dropped rows (else a separate kernel did, or none are due)
+  const uint8_t* block_mask;  // [B*Hkv][nb][nb] over 128-blocks of compacted (query, key), or null
+  int nb;
   Budgets kept;
 };
 
@@ -120,6 +122,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
   const int last_pos = min(K, (c + 1) * P2) - 1;
   const int n_kt = last_pos / 128 + 1;  // key tiles 0..n_kt-1
   const int32_t* pm = p.perm + (size_t)grp * L;
+  // Block-sparse composition: key tile kt is processed when the block mask
+  // enables it for the 128-block of either M tile's positions (both tiles lie in
+  // one block unless G = 1); every role walks the same list of active tiles, and
+  // a tile disabled for only one M tile is fully masked in that tile's softmax.
+  const uint8_t* bm = p.block_mask ? p.block_mask + (size_t)grp * p.nb * p.nb : nullptr;
+  const int qb0 = (c * P2) / 128, qb1 = (c * P2 + p.RP) / 128;
+  auto tile_on = [&](int t, int kt) -> bool { return bm == nullptr || bm[(t ? qb1 : qb0) * p.nb + kt] != 0; };
+  auto active = [&](int kt) -> bool { return tile_on(0, kt) || tile_on(1, kt); };
+  auto next_active = [&](int kt) -> int {
+    int x = kt + 1;
+    while (x < n_kt && !active(x)) ++x;
+    return x;
+  };
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -140,6 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_act = n_kt;  // active key tiles
+  if (bm != nullptr) {
+    n_act = 0;
+    for (int x0 = 0; x0 < n_kt; x0 += 32) n_act += __popc(__ballot_sync(0xffffffffu, x0 + lane < n_kt && active(x0 + lane)));
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 32 * kProducerWarps);  // every producer lane publishes its own copies
@@ -213,18 +233,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);   // group 1
     int committed = 2;  // groups 0, 1: Q tiles; group 2 + r: ring load r
     const int kv_row0 = (b * p.Hkv + g) * L;
-    int y_next = kv_row0 + load_pos(pm, min(my_row, K - 1), L, p.status);
+    int kt_load = next_active(-1);  // the active tile whose rows y_next holds
+    int y_next = kv_row0 + load_pos(pm, min(min(kt_load, n_kt - 1) * 128 + my_row, K - 1), L, p.status);
     int published = 0;  // ring loads published so far
     bool q_published = false;
-    for (int i = 0; i < 2 * n_kt; ++i) {
+    for (int i = 0; i < 2 * n_act; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int j = i >> 1;
       const int s = i % C::NS;
-      if ((i & 1) == 0) {  // K_j: tile j's rows become current, fetch tile j+1's indices
+      if ((i & 1) == 0) {  // K of an active tile: its rows become current, fetch the next active tile's
         __syncwarp();
         kvtab[my_row] = y_next;
         __syncwarp();
-        if (j + 1 < n_kt) y_next = kv_row0 + load_pos(pm, min((j + 1) * 128 + my_row, K - 1), L, p.status);
+        kt_load = next_active(kt_load);
+        if (kt_load < n_kt) y_next = kv_row0 + load_pos(pm, min(kt_load * 128 + my_row, K - 1), L, p.status);
       }
       if (i >= C::NS) {  // wait until load i - NS (same stage) has been consumed
         const bool got = mbar_wait(bar_empty(s), ((i / C::NS) - 1) & 1, p.wait_limit, abort_flag);
@@ -295,8 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           mma_bf16_ts(tmem + C::O_COL0 + t * D, tmem + (uint32_t)t * 128u + kk * 8,
                       sdesc_sw128(vbase + kk * 2048, 16384, 1024), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
       };
-      if (ok) ok = wait_load(0);
-      if (ok) {
+      if (ok && n_act > 0) ok = wait_load(0);
+      if (ok && n_act > 0) {
         tc_fence_after();
         qk(0, 0);
         tc_commit(bar_s(0));
@@ -304,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         tc_commit(bar_s(1));
         tc_commit(bar_empty(0));  // K_0 consumed once both QKs complete
       }
-      for (int j = 0; ok && j < n_kt; ++j) {
+      for (int j = 0; ok && j < n_act; ++j) {  // j counts active tiles
         const int iv = 2 * j + 1, ik_next = 2 * j + 2;
         if (!(ok = wait_load(iv))) break;
         for (int t = 0; t < 2 && ok; ++t) {
@@ -312,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           tc_fence_after();
           pv(t, iv, j > 0);
           if (t == 1) tc_commit(bar_empty(iv % C::NS));  // V_j consumed
-          if (j + 1 < n_kt) {
+          if (j + 1 < n_act) {
             if (t == 0 && !(ok = wait_load(ik_next))) break;
             tc_fence_after();
             qk(t, ik_next);
@@ -344,11 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     // The two softmax warpgroups run independently: while one is in its
     // latency-bound max pass the other keeps the exponential unit busy.  (Taking
     // strict turns on the whole softmax phase measured 8 % slower.)
-    for (int j = 0; j < n_kt; ++j) {
+    int kt = next_active(-1);  // key tile of active step j
+    for (int j = 0; j < n_act; ++j, kt = next_active(kt)) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s(t), j & 1, p.wait_limit, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      const int nvis = pos - j * 128 + 1;  // visible keys in this tile (causal)
+      // Visible keys in this tile: causal, and none when the block mask disables it for this M tile.
+      const int nvis = tile_on(t, kt) ? pos - kt * 128 + 1 : 0;
       // Only tiles on the diagonal hide keys from some rows (warp-uniform choice).
       const bool masked = __any_sync(0xffffffffu, nvis < 128);
       // Two passes over S_t, each in four 32-column chunks whose TMEM loads run one
@@ -394,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         }
         rescaled = j > 0 && __any_sync(0xffffffffu, need);
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t negm2 = f2_pack(-m_use, -m_use);
+        const float mref = m_use == -INFINITY ? 0.f : m_use;  // no visible key yet: P = 2^-inf = 0
+        const uint64_t negm2 = f2_pack(-mref, -mref);
         uint64_t accq[2] = {0ull, 0ull};
         // Pairs of chunks per iteration of a rolled loop: the loop edge keeps the
         // scheduler from interleaving all four chunks (which ran out of registers).
@@ -447,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       tc_fence_before();
       mbar_arrive(bar_p(t));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o(t), 0, p.wait_limit, abort_flag));
+    if (ok && n_act > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o(t), 0, p.wait_limit, abort_flag));
     if (!ok) {
       fail();
     } else {
@@ -455,11 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       const bool valid = pos < K;
       const int opos = valid ? load_pos(pm, pos, L, p.status) : 0;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + ((size_t)(b * p.Hq + g * p.G + hh) * L + opos) * D;
-      const float inv = 1.f / l;
+      const float inv = l > 0.f ? 1.f / l : 0.f;  // a row that saw no key (block mask) outputs zeros
 #pragma unroll
       for (int q4 = 0; q4 < D / 32; ++q4) {
         uint32_t v[32];
-        tmem_ld32(tO + q4 * 32, v);  // warp-collective: every lane loads, valid rows store
+        if (n_act > 0) {
+          tmem_ld32(tO + q4 * 32, v);  // warp-collective: every lane loads, valid rows store
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;  // no active key tile: O was never written
+        }
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
 #pragma unroll
@@ -501,7 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
 
 template <int D>
 cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                      const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st) {
+                      const Budgets& kept, void* out, uint32_t* status, bool accumulate, const uint8_t* block_mask,
+                      cudaStream_t st) {
   TcAttendParams prm;
   prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.k = static_cast<const __nv_bfloat16*>(k);
@@ -526,6 +556,8 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
   // The fused zero fill spreads the dropped rows over the attention CTAs; with
   // fewer of those than two per SM (small budgets) a separate full-grid zero
   // kernel writes them at HBM speed instead.
+  prm.block_mask = block_mask;
+  prm.nb = (d.L + 127) / 128;
   prm.zero_fill = 0;
   if (!accumulate) {
     if (nblk >= kFusedZeroMinCtas) {
@@ -546,9 +578,10 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
 }  // namespace
 
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                             const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st) {
-  return d.D == 64 ? launch_tc<64>(d, q, k, v, perm, kept, out, status, accumulate, st)
-                   : launch_tc<128>(d, q, k, v, perm, kept, out, status, accumulate, st);
+                             const Budgets& kept, void* out, uint32_t* status, bool accumulate,
+                             const uint8_t* block_mask, cudaStream_t st) {
+  return d.D == 64 ? launch_tc<64>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st)
+                   : launch_tc<128>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st);
 }
 
 }  // namespace tsa

@@ -52,11 +52,14 @@ cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kep
                           uint32_t* status, cudaStream_t st);
 cudaError_t launch_select_coverage(const Dims& d, const float* scores, double tau, int32_t* perm, int32_t* k_out,
                                    uint32_t* status, cudaStream_t st);
+// block_mask: optional [B*Hkv][nb][nb] bytes (nb = ceil(L/128)) over 128-blocks of
+// compacted (query, key) positions; null for plain causal attention.
 cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* perm, const Budgets& kept, void* out, uint32_t* status,
-                               bool accumulate, cudaStream_t st);
+                               bool accumulate, const uint8_t* block_mask, cudaStream_t st);
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                             const Budgets& kept, void* out, uint32_t* status, bool accumulate, cudaStream_t st);
+                             const Budgets& kept, void* out, uint32_t* status, bool accumulate,
+                             const uint8_t* block_mask, cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
 constexpr int kDriftMaxBlocks = 2048;  // drift partials held in its workspace

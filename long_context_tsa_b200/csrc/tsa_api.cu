@@ -127,15 +127,16 @@ tsa_status run_select(const Dims& d, const float* scores, const Budgets& kb, int
 }
 
 tsa_status run_attend(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
-                      const Budgets& kb, void* out, void* ws, cudaStream_t st, bool accumulate = false) {
+                      const Budgets& kb, void* out, void* ws, cudaStream_t st, bool accumulate = false,
+                      const uint8_t* block_mask = nullptr) {
   // The tensor-core kernel zero-fills the dropped rows itself (unless accumulating).
   if (d.dtype == TSA_BF16)
-    return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), accumulate, st));
+    return cuda_status(launch_attend_tc(d, q, k, v, perm, kb, out, status_word(ws), accumulate, block_mask, st));
   if (!accumulate) {
     const tsa_status s = cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), st));
     if (s != TSA_OK) return s;
   }
-  return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), accumulate, st));
+  return cuda_status(launch_attend_simt(d, q, k, v, perm, kb, out, status_word(ws), accumulate, block_mask, st));
 }
 
 __global__ void debug_wait_kernel(uint32_t* status, const uint32_t* flag, uint64_t limit) {
@@ -229,6 +230,21 @@ tsa_status tsa_attend_accumulate(const tsa_desc* desc, const void* q, const void
   Budgets kb;
   if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
   return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream), true);
+}
+
+tsa_status tsa_attend_block_sparse(const tsa_desc* desc, const void* q, const void* k, const void* v,
+                                   const int32_t* perm, const int32_t* budget_host, const uint8_t* block_mask,
+                                   void* out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(perm) || !aligned16(out) || !aligned16(ws) ||
+      block_mask == nullptr)
+    return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream), false, block_mask);
 }
 
 size_t tsa_drift_workspace_size(void) { return kDriftWsBytes; }

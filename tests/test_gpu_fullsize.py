@@ -10,10 +10,11 @@ import numpy as np
 import pytest
 import torch
 
+import long_context_tsa_b200 as T
 from long_context_tsa_b200 import inputs as I
 from oracle import tsa_oracle as O
 
-from .parity_util import Run, assert_dropped_rows_zero, assert_scores_close, compare_attend, host
+from .parity_util import Run, assert_dropped_rows_zero, assert_rows_close, assert_scores_close, compare_attend, host
 
 pytestmark = pytest.mark.gpu
 
@@ -71,3 +72,31 @@ def test_dense_keep_all_131072():
     r = Run(w, q, k, v)
     out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
     compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=8, seed=3)
+
+
+def test_block_sparse_131072():
+    # Block-sparse composition at the bench size: diagonal blocks, the first block
+    # column (sinks) and a seeded half of the other causal blocks.
+    w, q, k, v, qn, kn, vn = _setup("gqa_bf16_L131072", seed=4)
+    budgets = w.budgets()
+    perm = O.select(O.score(qn, kn, w.W).astype(np.float32), budgets)
+    nb = -(-w.L // 128)
+    rng = np.random.default_rng(5)
+    bm = (rng.random((w.B, w.Hkv, nb, nb)) < 0.5).astype(np.uint8)
+    bm[:, :, np.arange(nb), np.arange(nb)] = 1
+    bm[:, :, :, 0] = 1
+    r = Run(w, q, k, v)
+    r.out.fill_(float("nan"))
+    T.tsa_attend_block_sparse(r.desc, q, k, v, torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets,
+                              torch.from_numpy(bm).to(DEV), r.out, r.ws)
+    assert r.status() == 0
+    kept = O.clamp_budgets(budgets, w.L)
+    rs = np.random.default_rng(6)
+    for h in range(0, w.Hq, 3):
+        g = h // w.G
+        K = int(kept[g])
+        rows = np.unique(np.concatenate([rs.choice(K, 24, replace=False), [0, K - 1]]))
+        ora = O.attend_rows(qn, kn, vn, perm[0, g], K, 0, h, w.G, rows, block_mask_bg=bm[0, g])
+        pos = torch.from_numpy(perm[0, g, rows]).to(DEV)
+        assert_rows_close(host(r.out[0, h].index_select(0, pos)), ora, w.dtype, f"h={h}")
+    assert_dropped_rows_zero(r.out, torch.from_numpy(perm).to(DEV), budgets, w.G)

@@ -224,3 +224,55 @@ def test_attend_accumulate_scatter_adds(w):
             assert_rows_close(got[b, h, rows], ora[b, h, rows], w.dtype, f"b={b} h={h}")
             drop = torch.from_numpy(perm[b, g, K:]).to(DEV)
             assert torch.equal(out[b, h].index_select(0, drop), base[b, h].index_select(0, drop)), (b, h)
+
+
+def _block_mask(w, density, seed, kill_first_diag=False):
+    nb = -(-w.L // 128)
+    rng = np.random.default_rng(seed)
+    bm = (rng.random((w.B, w.Hkv, nb, nb)) < density).astype(np.uint8)
+    idx = np.arange(nb)
+    bm[:, :, idx, idx] = 1  # the diagonal on ...
+    if kill_first_diag:
+        bm[:, 0, 0, 0] = 0  # ... except block 0 of group 0: its rows see no key at all
+    return bm
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("density", [0.0, 0.4, 1.0])
+def test_attend_block_sparse_matches_oracle(w, density):
+    q, k, v, qn, kn, vn = _inputs(w, seed=12)
+    rng = np.random.default_rng(13)
+    budgets = [int(x) for x in rng.integers(1, w.L + 1, size=w.B * w.Hkv)]
+    perm = O.select(rng.random((w.B, w.Hkv, w.L)).astype(np.float32), budgets)
+    bm = _block_mask(w, density, seed=14, kill_first_diag=density == 0.4)
+    r = Run(w, q, k, v)
+    r.out.fill_(float("nan"))
+    T.tsa_attend_block_sparse(r.desc, q, k, v, torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets,
+                              torch.from_numpy(bm).to(DEV), r.out, r.ws)
+    assert r.status() == 0
+    ora = O.attend_block_sparse(qn, kn, vn, perm, budgets, bm)
+    got = host(r.out)
+    kept = O.clamp_budgets(budgets, w.L)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            g = h // w.G
+            rows = perm[b, g, :int(kept[b * w.Hkv + g])]
+            assert_rows_close(got[b, h, rows], ora[b, h, rows], w.dtype, f"b={b} h={h}")
+    assert_dropped_rows_zero(r.out, torch.from_numpy(perm).to(DEV), budgets, w.G)
+    if density == 0.4:  # rows with no visible key are exact zeros
+        rows0 = perm[0, 0, :min(128, int(kept[0]))]
+        assert np.all(got[0, :w.G][:, rows0] == 0.0)
+
+
+def test_attend_block_sparse_full_mask_equals_attend():
+    w = SMALL[3]
+    q, k, v, qn, kn, vn = _inputs(w, seed=15)
+    budgets = w.budgets()
+    perm_t = torch.from_numpy(O.select(O.score(qn, kn, w.W).astype(np.float32), budgets).astype(np.int32)).to(DEV)
+    r = Run(w, q, k, v)
+    dense = r.attend(perm_t, budgets).clone()
+    nb = -(-w.L // 128)
+    ones = torch.ones((w.B, w.Hkv, nb, nb), dtype=torch.uint8, device=DEV)
+    T.tsa_attend_block_sparse(r.desc, q, k, v, perm_t, budgets, ones, r.out, r.ws)
+    assert r.status() == 0
+    assert torch.equal(r.out, dense)  # the same kernel path, bit for bit
