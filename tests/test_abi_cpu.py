@@ -111,3 +111,46 @@ def test_status_strings(lib):
     for code in range(7):
         assert N.tsa_status_string(code)
     assert N.tsa_status_string(99) == "unknown status"
+
+
+def test_next_row_calls_reject_before_launch(lib):
+    d = desc()
+    b = N._budgets([4096] * 8)
+    bad_b = N._budgets([4096] * 7 + [0])
+    inv, wsz = N.STATUS["TSA_ERR_INVALID_ARG"], N.STATUS["TSA_ERR_WORKSPACE"]
+    # Scatter-add attention: same rules as tsa_attend.
+    assert lib.tsa_attend_accumulate(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, bad_b, FAKE, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_attend_accumulate(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, b, FAKE + 2, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_attend_accumulate(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, b, FAKE, FAKE, 16, None) == wsz
+    # Block-sparse attention: a mask is required.
+    assert lib.tsa_attend_block_sparse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, b, None, FAKE, FAKE, 1 << 20,
+                                       None) == inv
+    assert lib.tsa_attend_block_sparse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, bad_b, FAKE, FAKE, FAKE, 1 << 20,
+                                       None) == inv
+    # Coverage selection: tau in [0, 1], a budget output, the usual pointer rules.
+    for tau in (-0.5, 1.01, float("nan"), float("inf")):
+        assert lib.tsa_select_coverage(ctypes.byref(d), FAKE, tau, FAKE, FAKE, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_select_coverage(ctypes.byref(d), FAKE, 0.1, FAKE, None, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_select_coverage(ctypes.byref(d), FAKE, 0.1, FAKE, FAKE + 2, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_select_coverage(ctypes.byref(d), FAKE, 0.1, FAKE, FAKE, FAKE, 16, None) == wsz
+    out = (ctypes.c_int32 * 8)()
+    assert lib.tsa_forward_coverage(ctypes.byref(d), FAKE, FAKE, FAKE, 64, 2.0, out, None, None, FAKE, FAKE,
+                                    1 << 40, None) == inv
+    assert lib.tsa_forward_coverage(ctypes.byref(d), FAKE, FAKE, FAKE, 64, 0.1, None, None, None, FAKE, FAKE,
+                                    1 << 40, None) == inv
+    assert lib.tsa_forward_coverage(ctypes.byref(d), FAKE, FAKE, FAKE, 64, 0.1, out, None, None, FAKE, FAKE,
+                                    256, None) == wsz
+
+
+def test_binding_checks_block_mask_shape():
+    import torch
+
+    import long_context_tsa_b200 as T
+
+    d = desc(L=1000)
+    wrong = torch.zeros((1, 8, 7, 7), dtype=torch.uint8)  # nb = 8 for L = 1000
+    with pytest.raises(ValueError):
+        T.tsa_attend_block_sparse(d, None, None, None, None, [1] * 8, wrong, None, torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        T.tsa_attend_block_sparse(d, None, None, None, None, [1] * 8, torch.zeros((1, 8, 8, 8)), None,
+                                  torch.zeros(16, dtype=torch.uint8))
