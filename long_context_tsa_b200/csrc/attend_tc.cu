@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
           continue;
         }
         uint4* row = ob + (size_t)pos * CPR;
-        for (int hh = 0; hh < p.G; ++hh) row[hh * head_stride] = zero;
+        // Streaming (evict-first) stores: the zeros must not push the K/V rows other CTAs still read out of L2.
+        for (int hh = 0; hh < p.G; ++hh) __stcs(row + hh * head_stride, zero);
       }
     }
   } else if (warp == kMmaWarp) {
