@@ -54,8 +54,15 @@ struct SelectArgs {
 };
 
 __device__ __forceinline__ uint64_t token_mass(float s, float mass_scale) {
-  // fmaxf drops NaN; scaling by a power of two is exact; truncation is floor here.
-  return __float2ull_rz(fminf(fmaxf(s, 0.f), 256.f) * mass_scale);
+  // fmaxf drops NaN; scaling by a power of two is exact, so v = s * 2^S is the
+  // exact real value, and floor(v) is its significand shifted by its exponent
+  // (integer bit operations; a float-to-64-bit conversion is much slower).
+  const float v = fminf(fmaxf(s, 0.f), 256.f) * mass_scale;
+  const uint32_t bits = __float_as_uint(v);
+  const int k = (int)(bits >> 23) - 150;  // v = (1.f23 significand as integer) * 2^k for normal v
+  if ((bits >> 23) == 0u || k <= -24) return 0u;  // zero, subnormal or below 1: floor is 0
+  const uint64_t sig = (bits & 0x7FFFFFu) | 0x800000u;
+  return k >= 0 ? sig << k : sig >> -k;
 }
 
 __device__ __forceinline__ float key_to_float(uint32_t key) {
@@ -140,7 +147,9 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   __shared__ uint32_t dig_warp[8];
   __shared__ uint32_t sh_digit, sh_above;
   __shared__ uint32_t cnt[2];  // this slice's (#key > T, #key == T)
-  __shared__ uint64_t histm[2][256];  // coverage mode: mass per digit
+  // Coverage mode: mass per digit as 32-bit halves (64-bit shared atomics are
+  // much slower): lo wraps modulo 2^32 and every wrap adds one to hi.
+  __shared__ uint32_t histml[2][256], histmh[2][256];
   __shared__ uint64_t dig_warp_m[8];
   __shared__ uint64_t sh_mass, sh_mabove;
 
@@ -166,10 +175,12 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
       for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         uint32_t* hc = hist[pass & 1];
-        uint64_t* hm = histm[pass & 1];
+        uint32_t* hml = histml[pass & 1];
+        uint32_t* hmh = histmh[pass & 1];
         if (tid < 256) {
           hc[tid] = 0u;
-          hm[tid] = 0u;
+          hml[tid] = 0u;
+          hmh[tid] = 0u;
         }
         __syncthreads();
         for (int i = lo + tid; i < hi; i += kThreads) {
@@ -179,7 +190,13 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
             const uint32_t dg = (key >> shift) & 255u;
             atomicAdd(&hc[dg], 1u);
             const uint64_t m = token_mass(f, a.mass_scale);
-            if (m) atomicAdd(reinterpret_cast<unsigned long long*>(&hm[dg]), (unsigned long long)m);
+            const uint32_t mlo = (uint32_t)m;
+            uint32_t mhi = (uint32_t)(m >> 32);
+            if (mlo) {
+              const uint32_t old = atomicAdd(&hml[dg], mlo);
+              mhi += (old + mlo < old);  // the low word wrapped
+            }
+            if (mhi) atomicAdd(&hmh[dg], mhi);
           }
         }
         cluster.sync();
@@ -190,7 +207,8 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
           uint64_t totm = 0u;
           for (int r = 0; r < kClusterCtas; ++r) {
             totc += cluster.map_shared_rank(hc, r)[255 - tid];
-            totm += cluster.map_shared_rank(hm, r)[255 - tid];
+            totm += ((uint64_t)cluster.map_shared_rank(hmh, r)[255 - tid] << 32) +
+                    cluster.map_shared_rank(hml, r)[255 - tid];
           }
           uint64_t Sm;
           uint32_t Sc;
