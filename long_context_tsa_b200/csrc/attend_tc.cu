@@ -87,7 +87,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_IDX + 3 * 128 * 4;
   // barriers: q, full[NS], empty[NS], s[2], p[2], o[2], teardown; then tmem slot, abort flag
   static constexpr int NBAR = 1 + 2 * NS + 6 + 1;
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int OFF_ZERO = (OFF_BAR + NBAR * 8 + 16 + 15) / 16 * 16;  // one row of zeros (bulk-copy source)
+  static constexpr int SMEM = OFF_ZERO + D * 2 + 1024;  // + alignment slack
   static constexpr int CPR = D / 8;    // 16-byte chunks per row
   static constexpr int RPI = 32 / CPR;  // rows per warp-wide copy instruction
   static constexpr int DEFER = 2;       // copy groups left in flight before a group is published
@@ -273,22 +274,25 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     if (U > 0) {
       const int nc = (K + P2 - 1) / P2;  // CTAs of this group
       const int lo = (int)((long long)U * c / nc), hi = (int)((long long)U * (c + 1) / nc);
+      // Each dropped row of each query head is one bulk (TMA) copy of a shared-memory
+      // row of zeros: the copy engine moves the bytes, the warps only issue them
+      // (plain 16-byte stores from these warps measured 2 % slower overall).
       constexpr int CPR = D * 2 / 16;  // 16-byte chunks per row
-      constexpr int RPI = 32 / CPR;    // rows per warp instruction
-      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-      uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)(b * p.Hq + g * p.G) * L * D) +
-                  lane % CPR;
-      const size_t head_stride = (size_t)L * CPR;  // in 16-byte chunks
-      for (int u = lo + (warp - kZeroWarp0) * RPI + lane / CPR; u < hi; u += RPI * kZeroWarps) {
+      const uint32_t szero = base + C::OFF_ZERO;
+      const int zt = (warp - kZeroWarp0) * 32 + lane;  // 0 .. 32 * kZeroWarps - 1
+      if (zt < CPR) st_shared_v4(szero + 16 * zt, 0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();  // the zeros are visible to the copy engine ...
+      named_sync(3u, 32u * kZeroWarps);  // ... before any zero warp copies them
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.out) + (size_t)(b * p.Hq + g * p.G) * L * D;
+      for (int u = lo + zt; u < hi; u += 32 * kZeroWarps) {
         const int pos = pm[K + u];
         if ((unsigned)pos >= (unsigned)L) {
           record_status(p.status, TSA_ERR_DEVICE_BOUNDS);
           continue;
         }
-        uint4* row = ob + (size_t)pos * CPR;
-        // Streaming (evict-first) stores: the zeros must not push the K/V rows other CTAs still read out of L2.
-        for (int hh = 0; hh < p.G; ++hh) __stcs(row + hh * head_stride, zero);
+        for (int hh = 0; hh < p.G; ++hh) bulk_copy_s2g(ob + ((size_t)hh * L + pos) * D, szero, D * 2);
       }
+      bulk_commit_wait_all();  // the source row stays valid and every copy is done before the CTA exits
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer

@@ -289,6 +289,19 @@ __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Bulk copy (copy engine) of `bytes` from shared memory to global memory; both
+// addresses 16-byte aligned, `bytes` a multiple of 16.  Tracked by bulk groups.
+__device__ __forceinline__ void bulk_copy_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(gdst)),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+// Commit this thread's bulk copies and wait until all of them have completed.
+__device__ __forceinline__ void bulk_commit_wait_all() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
