@@ -100,3 +100,28 @@ def test_block_sparse_131072():
         pos = torch.from_numpy(perm[0, g, rows]).to(DEV)
         assert_rows_close(host(r.out[0, h].index_select(0, pos)), ora, w.dtype, f"h={h}")
     assert_dropped_rows_zero(r.out, torch.from_numpy(perm).to(DEV), budgets, w.G)
+
+
+def test_accumulate_8192_many_items_per_cta():
+    # 512 work items on at most 148 persistent CTAs: every kept row must be added
+    # exactly once (a repeated item would add its rows twice), dropped rows untouched.
+    w, q, k, v, qn, kn, vn = _setup("gqa_bf16_L8192", seed=6)
+    budgets = w.budgets()
+    perm = O.select(np.random.default_rng(7).random((w.B, w.Hkv, w.L)).astype(np.float32), budgets)
+    base = torch.randn(q.shape, generator=torch.Generator().manual_seed(8)).to(q.dtype).to(DEV)
+    out = base.clone()
+    r = Run(w, q, k, v)
+    T.tsa_attend_accumulate(r.desc, q, k, v, torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets, out, r.ws)
+    assert r.status() == 0
+    kept = O.clamp_budgets(budgets, w.L)
+    bn = host(base)
+    rs = np.random.default_rng(9)
+    for h in range(w.Hq):
+        g = h // w.G
+        K = int(kept[g])
+        rows = np.unique(np.concatenate([rs.choice(K, 32, replace=False), [0, K - 1]]))
+        ora = bn[0, h, perm[0, g, rows]] + O.attend_rows(qn, kn, vn, perm[0, g], K, 0, h, w.G, rows)
+        pos = torch.from_numpy(perm[0, g, rows]).to(DEV)
+        assert_rows_close(host(out[0, h].index_select(0, pos)), ora, w.dtype, f"h={h}")
+        drop = torch.from_numpy(perm[0, g, K:]).to(DEV)
+        assert torch.equal(out[0, h].index_select(0, drop), base[0, h].index_select(0, drop))
