@@ -14,8 +14,12 @@
 //           c_r = m_r + log2 Z_r combined over all splits,
 //           score[j] = sum_r 2^(x_rj - c_r)  -- one thread per key, no
 //           cross-thread reduction.
-// Warp roles (320 threads): warps 0-3 and 4-7 read TMEM (two warpgroups),
-// warp 8 loads (TMA), warp 9 issues tcgen05.mma.  Bounded waits throughout.
+// Warp roles (576 threads): warps 0-15 read TMEM (four warpgroups; each
+// thread takes half of its TMEM row's columns, so every SM sub-partition has
+// four reader warps to hide the exponential unit's latency), warp 16 loads
+// (TMA), warp 17 issues tcgen05.mma.  Pass 1 merges the two column halves of
+// each row's (m, Z); pass 2 adds the two halves of each key's sum into the
+// scores, which pass 1 zeroed.  Bounded waits throughout.
 #include <cuda.h>
 #include <math.h>
 
@@ -30,9 +34,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 576;
+constexpr int kReaders = 512;  // warps 0-15: four warpgroups read TMEM
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr uint32_t kTeardownPolls = 1u << 26;
 
 struct ScoreTcParams {
@@ -54,8 +59,8 @@ struct SCfg {
   static constexpr int OFF_QW = 0;
   static constexpr int OFF_K = QW_BYTES;
   static constexpr int OFF_CST = OFF_K + NS * KT_BYTES;  // pass 2: Mp floats
-  static constexpr int OFF_RED = OFF_CST + 256 * 4;      // pass 1, RH == 1: 2 x 128 floats
-  static constexpr int OFF_BAR = OFF_RED + 256 * 4;
+  static constexpr int OFF_RED = OFF_CST + 256 * 4;      // pass 1: partial (m, Z) of the other warpgroups
+  static constexpr int OFF_BAR = OFF_RED + 4 * 256 * 4;
   // barriers: q, full[NS], empty[NS], sfull[2], sfree[2], teardown
   static constexpr int NBAR = 1 + 2 * NS + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_sfull(i), 1);
-      mbar_init(bar_sfree(i), PASS == 1 ? 256 : 128);
+      mbar_init(bar_sfree(i), PASS == 1 ? kReaders : kReaders / 2);
     }
     mbar_init(bar_td, 1);
     *abort_flag = 0;
@@ -232,32 +237,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ TMEM readers
-    const int wg = warp >> 2;
+    const int wg = warp >> 2;       // 0..3
+    const int a = wg & 1;           // row half (pass 1, RH == 2) or tile parity
+    const int ch = wg >> 1;         // column half of the TMEM row this thread reads
     const int rl = threadIdx.x & 127;  // TMEM lane of this thread
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
     if (PASS == 1) {
-      const int r = RH == 2 ? wg * 128 + rl : rl;  // window row
+      const int r = RH == 2 ? a * 128 + rl : rl;  // window row
       const int pos = L - p.W + (r % p.W);
       const bool row_ok = r < p.M;
+      // Pass 2 adds its two column halves into the scores: start them at zero.
+      for (int j = j0 + threadIdx.x; j < j1; j += kReaders) p.scores[(size_t)grp * L + j] = 0.f;
       float m = -INFINITY, z = 0.f;
       for (int i = 0; i < nstep; ++i) {
         const int bf = i & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (i >> 1) & 1, p.wait_limit, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        const int u = RH == 2 ? i : 2 * i + wg;
-        uint32_t v[128];
-        if (u < nt) tmem_ld128(tmem + lane_off + bf * 256 + wg * 128, v);
+        const int u = RH == 2 ? i : 2 * i + a;
+        uint32_t v[64];
+        if (u < nt) {
+          const uint32_t ta = tmem + lane_off + bf * 256 + a * 128 + ch * 64;
+          tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld32(*reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_wait_ld32(*reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        }
         tc_fence_before();
         mbar_arrive(bar_sfree(bf));
         if (u < nt) {
-          const int kbase = j0 + 128 * u;
-          const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this tile
-          const bool masked = __any_sync(0xffffffffu, lim < 128);
+          const int kbase = j0 + 128 * u + 64 * ch;
+          const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this half tile
+          const bool masked = __any_sync(0xffffffffu, lim < 64);
           if (masked) {
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
+            for (int e = 0; e < 64; ++e)
               if (e >= lim) v[e] = 0xff800000u;  // -inf
           }
           // z is kept relative to a per-row reference m: any reference gives the
@@ -268,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t negm2 = f2_pack(-ref, -ref), sc2 = f2_pack(p.scale_log2, p.scale_log2);
             uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int e2 = 0; e2 < 64; ++e2) {
+            for (int e2 = 0; e2 < 32; ++e2) {
               float t0, t1;
               f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, negm2), t0, t1);
               a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(ex2_approx(t0), ex2_approx(t1)));
@@ -287,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
 #pragma unroll
-            for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+            for (int e = 8; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
             const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
             if (exact && mt > -INFINITY) {
@@ -301,35 +316,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           z += st;
         }
       }
+      // Merge the partial (m, Z) of the warpgroups that saw the same rows: both
+      // column halves, and for RH == 1 also both tile parities.  The named
+      // barrier is reached by all reader threads whatever happened above.
+      const int slot = RH == 2 ? (ch * 2 + a) : wg;  // 4 slots of 128 (RH == 1) or 2 x 2 (RH == 2)
+      red[slot * 128 + rl] = m;
+      red[512 + slot * 128 + rl] = z;
+      asm volatile("bar.sync 1, %0;" ::"n"(kReaders) : "memory");
       if (!ok) fail();
-      float* pp = p.part + ((size_t)grp * p.nsplit + split) * Mp * 2;
-      if (RH == 2) {
-        if (ok) {
-          pp[r] = m;
-          pp[Mp + r] = z;
+      const bool writer = RH == 2 ? (ch == 0) : (wg == 0);
+      if (writer && !*abort_flag) {
+        constexpr int NSRC = RH == 2 ? 2 : 4;  // partials per row
+        float ms[NSRC], zs4[NSRC];
+#pragma unroll
+        for (int i = 0; i < NSRC; ++i) {
+          const int sl = RH == 2 ? (i * 2 + a) : i;
+          ms[i] = red[sl * 128 + rl];
+          zs4[i] = red[512 + sl * 128 + rl];
         }
-      } else {
-        // Both warpgroups saw the same rows on alternate key tiles: merge.  The
-        // named barrier is reached by all 256 threads whatever happened above.
-        if (wg == 1) {
-          red[rl] = m;
-          red[128 + rl] = z;
+        float mn = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NSRC; ++i) mn = fmaxf(mn, ms[i]);
+        float zz = 0.f;
+        if (mn > -INFINITY) {
+#pragma unroll
+          for (int i = 0; i < NSRC; ++i)
+            if (ms[i] > -INFINITY) zz += zs4[i] * ex2_approx(ms[i] - mn);
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (wg == 0 && !*abort_flag) {
-          const float m2 = red[rl], z2 = red[128 + rl];
-          const float mn = fmaxf(m, m2);
-          float zz = 0.f;
-          if (mn > -INFINITY)
-            zz = (m > -INFINITY ? z * ex2_approx(m - mn) : 0.f) + (m2 > -INFINITY ? z2 * ex2_approx(m2 - mn) : 0.f);
-          pp[r] = mn;
-          pp[Mp + r] = zz;
-        }
+        float* pp = p.part + ((size_t)grp * p.nsplit + split) * Mp * 2;
+        pp[r] = mn;
+        pp[Mp + r] = zz;
       }
     } else {
       // Combine the row partials of every split: c_r = m_r + log2 Z_r.
       const float* pbase = p.part + (size_t)grp * p.nsplit * Mp * 2;
-      for (int r = threadIdx.x; r < Mp; r += 256) {
+      for (int r = threadIdx.x; r < Mp; r += kReaders) {
         float mx = -INFINITY;
         for (int s = 0; s < p.nsplit; ++s) mx = fmaxf(mx, pbase[(size_t)s * Mp * 2 + r]);
         float zs = 0.f;
@@ -341,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cst[r] = (r < p.M && mx > -INFINITY) ? -(mx + log2f(zs)) : -INFINITY;  // -c_r
       }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kReaders) : "memory");
       float* out = p.scores + (size_t)grp * L;
-      for (int u = wg; u < nt; u += 2) {
+      constexpr int HC = Mp / 2;  // columns (window rows) of this thread's half
+      for (int u = a; u < nt; u += 2) {
         const int bf = u & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (u >> 1) & 1, p.wait_limit, abort_flag));
         if (!ok) break;
@@ -354,10 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool tail = __any_sync(0xffffffffu, key >= L - p.W);
         float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int q4 = 0; q4 < Mp / 32; ++q4) {
+        for (int q4 = 0; q4 < HC / 32; ++q4) {
+          const int col0 = ch * HC + q4 * 32;  // first window row of this chunk
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + bf * 256 + q4 * 32, v);
-          const float* nc = cst + q4 * 32;
+          tmem_ld32(tmem + lane_off + bf * 256 + col0, v);
+          const float* nc = cst + col0;
           if (!tail) {
             const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
             uint64_t a2[2] = {0ull, 0ull};
@@ -378,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const int col = q4 * 32 + e;
+              const int col = col0 + e;
               const float pe = ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, nc[e]));
               acc4[e & 3] += (key > L - p.W + (col % p.W)) ? 0.f : pe;
             }
@@ -387,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
         tc_fence_before();
         mbar_arrive(bar_sfree(bf));
-        if (key < j1) out[key] = acc;
+        // Two column halves per key: 0 + h0 + h1 is the same in either order.
+        if (key < j1) atomicAdd(out + key, acc);
       }
       if (!ok) fail();
     }
