@@ -84,6 +84,31 @@ def block_sparse_flops(w, budgets, bm) -> float:
     return total
 
 
+def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: str):
+    """The step's other kernels against their own bounds.
+
+    score: the exponential unit (16 ex2 per clock per SM; both passes exponentiate
+    every (window row, key) logit once); select: HBM, on its algorithmic bytes
+    (scores read once, the permutation written once), which it cannot approach
+    because it is latency-bound (64 CTAs, cluster barriers between radix passes)."""
+    sms, mhz = 148, 1965.0
+    if torch.cuda.is_available():
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+    exps = 2.0 * w.B * w.Hkv * w.G * w.W * w.L
+    mufu_peak = 16.0 * sms * mhz * 1e6
+    a_score = exps / (t_score_ms * 1e-3)
+    sel_bytes = 2.0 * 4 * w.B * w.Hkv * w.L
+    a_sel = sel_bytes / (t_select_ms * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    return [
+        {"kernel": "score_tc (2 passes)", "bound": "alu", "achieved": a_score / 1e12, "peak": mufu_peak / 1e12,
+         "unit": "Tex2/s", "frac": a_score / mufu_peak,
+         "peak_source": f"16 ex2/clk/SM x {sms} SMs x {mhz:.0f} MHz (max SM clock)"},
+        {"kernel": "select_radix", "bound": "hbm", "achieved": a_sel, "peak": hbm, "unit": "GB/s",
+         "frac": a_sel / hbm, "peak_source": f"hbm_gbs ({peak_src})", "note": "latency-bound: 64 CTAs, cluster barriers between 4 radix passes"},
+    ]
+
+
 def rank_seed(rank: int) -> int:
     """Each rank runs its own independent layer (weak scaling): inputs seeded by rank."""
     return rank
@@ -428,6 +453,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"bf16_tflops ({peak_src})",
                      "kernel": "attend_tc (tsa_attend: gather + attention + scatter + zero fill)",
                      "traffic_source": traffic_src},
+        "rooflines_other": other_rooflines(w, t_score, t_select, peaks, peak_src),
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
