@@ -28,7 +28,9 @@
  * - Every tensor pointer is DEVICE memory owned by the caller, 16-byte aligned.
  *   The library allocates nothing, frees nothing and does not synchronise in
  *   the compute calls: work is enqueued on `stream` (a cudaStream_t passed as
- *   void*, NULL = legacy default stream) and the call returns.
+ *   void*, NULL = legacy default stream) and the call returns.  The documented
+ *   exceptions are tsa_forward_host (host buffers, copies on the stream) and
+ *   tsa_forward_coverage (one synchronisation to bring the chosen budgets back).
  * - `budget_host` is a HOST array of B*Hkv int32 kept-token counts, one per
  *   (batch, KV head), read during the call (grid planning needs it).  A budget
  *   <= 0 is TSA_ERR_INVALID_ARG; a budget > L is clamped to L, as [P1] Step 3
@@ -42,7 +44,7 @@
  *   are recorded in the workspace status word and reported by
  *   tsa_check_status().
  * - Supported: D in {64, 128}; Hq % Hkv == 0; G = Hq/Hkv in {1,2,4,8,16};
- *   1 <= window <= L; G*window <= 256; B*Hq*L < 2^31.
+ *   1 <= window <= L; G*window <= 256; B*Hq*L < 2^31; B*Hkv <= 1024.
  *   bf16 runs on tcgen05 tensor-core kernels, f32 on exact SIMT kernels.
  *   There is no CPU path.
  */
