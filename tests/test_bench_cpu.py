@@ -1,0 +1,51 @@
+"""Host-side helpers of bench.py: the flop and byte counts behind the reported
+rooflines (no GPU needed)."""
+
+import numpy as np
+
+import bench
+from long_context_tsa_b200 import inputs as I
+
+
+def test_block_sparse_flops_reduce_to_the_causal_count():
+    w = I.WORKLOADS["gqa_bf16_L8192"]
+    budgets = w.budgets()
+    nb = -(-w.L // 128)
+    ones = np.ones((w.B, w.Hkv, nb, nb), dtype=np.uint8)
+    assert bench.block_sparse_flops(w, budgets, ones) == bench.attend_flops(w, budgets)
+
+
+def test_block_sparse_flops_diagonal_blocks_closed_form():
+    w = I.custom(Hq=8, Hkv=2, L=1000, D=128, dtype="bf16", W=16)
+    budgets = [300, 1000]
+    nb = -(-w.L // 128)
+    diag = np.broadcast_to(np.eye(nb, dtype=np.uint8), (1, 2, nb, nb)).copy()
+    want = 0.0
+    for K in budgets:
+        for blk in range(0, K, 128):
+            n = min(128, K - blk)
+            want += w.G * 4.0 * w.D * n * (n + 1) / 2
+    assert bench.block_sparse_flops(w, budgets, diag) == want
+
+
+def test_block_mask_for_keeps_diagonal_and_sinks():
+    w = I.WORKLOADS["gqa_bf16_L8192"]
+    bm = bench.block_mask_for(w, 0.3)
+    nb = -(-w.L // 128)
+    assert bm.shape == (w.B, w.Hkv, nb, nb) and bm.dtype == np.uint8
+    assert np.all(bm[:, :, np.arange(nb), np.arange(nb)] == 1)
+    assert np.all(bm[:, :, :, 0] == 1)
+    frac = bm[:, :, 1:, 1:].mean()
+    assert 0.25 < frac < 0.4  # roughly the requested density off the forced blocks
+
+
+def test_other_rooflines_counts():
+    w = I.WORKLOADS["gqa_bf16_L131072"]
+    r = bench.other_rooflines(w, 0.19, 0.031, {"hbm_gbs": 6450.3}, "measured")
+    score, select = r
+    # 2 passes x (B x Hkv) groups x (G x W) window rows x L keys exponentials
+    assert abs(score["achieved"] * 1e12 * 0.19e-3 - 2 * 8 * 4 * 64 * 131072) < 1e3
+    assert score["bound"] == "alu" and 0 < score["frac"] < 1
+    # scores read once and the permutation written once: 8 bytes per key per group
+    assert abs(select["achieved"] * 1e9 * 0.031e-3 - 8 * 8 * 131072) < 1.0
+    assert select["bound"] == "hbm" and 0 < select["frac"] < 1
