@@ -276,6 +276,9 @@ TSA_API void tsa_debug_set_wait_limit(uint64_t polls);
 /* Number of kernels this library has launched in this process (all devices). */
 TSA_API uint64_t tsa_debug_launch_count(void);
 TSA_API tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream);
+/* y = 2^x through the FMA-pipe exponential the scoring kernel uses for one
+ * pair of values in three (device arrays of n floats, n even, 16-byte aligned). */
+TSA_API tsa_status tsa_debug_exp2(const float* x, float* y, int32_t n, void* stream);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,7 @@ EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
-            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse")
+            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2")
 
 
 class TsaDesc(ctypes.Structure):
@@ -59,6 +59,7 @@ _SIGS = {
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_debug_exp2": (ctypes.c_int, [_P, _P, _I32, _P]),
     "tsa_attend_block_sparse": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_select_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, ctypes.c_double, _P, _P, _P, _SZ, _P]),
     "tsa_forward_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P,
@@ -254,3 +255,8 @@ def tsa_attend_block_sparse(desc, q, k, v, perm, budgets, block_mask, out, ws, s
     _check(lib().tsa_attend_block_sparse(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
                                          _ptr(block_mask), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "tsa_attend_block_sparse")
+
+
+def tsa_debug_exp2(x, y, stream=None):
+    """y = 2^x through the library's FMA-pipe exponential (testing hook)."""
+    _check(lib().tsa_debug_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "tsa_debug_exp2")

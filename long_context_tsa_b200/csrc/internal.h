@@ -67,6 +67,7 @@ constexpr size_t kDriftWsBytes = 256 + sizeof(double) * kDriftMaxBlocks;
 int drift_grid(int64_t rows);
 cudaError_t launch_drift(int64_t rows, int hidden, int dtype, const void* a, const void* b, float* row_cos,
                          double* drift, void* ws, cudaStream_t st);
+cudaError_t launch_debug_exp2(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_debug_wait(uint32_t* status, uint32_t* flag, uint64_t limit, cudaStream_t st);
 
 }  // namespace tsa

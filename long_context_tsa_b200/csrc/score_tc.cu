@@ -34,6 +34,52 @@ namespace {
 
 using namespace tc;
 
+// ---- 2^t on the FMA pipe, for part of the column-sum exponentials ----
+//
+// The exponential unit (16 results per clock per SM) bounds both passes, so one
+// pair in three of pass 2's exponentials is computed with FMA-pipe arithmetic
+// instead (measured 6 % faster for the score).  Written from the math:
+// t = j + f with j = floor(t) and f in [0, 1); 2^f by a degree-4 polynomial
+// p(f) = 1 + f (c1 + f (c2 + f (c3 + f c4))) whose coefficients were fitted to
+// 2^f on [0, 1) by iteratively reweighted least squares on the relative error
+// (max relative error 3.0e-6 when evaluated in float32); 2^j by adding j to the
+// exponent field.  floor(t) comes from one add of 1.5 * 2^23 rounded toward
+// -infinity, whose low mantissa bits then hold j (the bits of 1.5 * 2^23 shift
+// out of the exponent field).  t is clamped to >= -126 so the result stays a
+// normal float: values below 2^-126 come out as 2^-126 instead of smaller, an
+// absolute error below 1.2e-38 per term.  Valid for t < 128 (pass 2 has t <= 0).
+__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ void ex2_fma_pair(float t0, float t1, float& p0, float& p1) {
+  const uint64_t magic = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
+  const uint64_t tt = f2_pack(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
+  const uint64_t y = f2_add_rm(tt, magic);
+  const uint64_t fr = f2_sub(tt, f2_sub(y, magic));
+  uint64_t q = f2_fma(f2_pack(0.013426822610199451f, 0.013426822610199451f), fr,
+                      f2_pack(0.052243269979953766f, 0.052243269979953766f));
+  q = f2_fma(q, fr, f2_pack(0.2412789911031723f, 0.2412789911031723f));
+  q = f2_fma(q, fr, f2_pack(0.6930451989173889f, 0.6930451989173889f));
+  q = f2_fma(q, fr, f2_pack(1.f, 1.f));
+  float q0, q1, y0, y1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(y, y0, y1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(y0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
+}
+
+__global__ void debug_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) ex2_fma_pair(x[i], x[i + 1], y[i], y[i + 1]);
+}
+
 constexpr int kThreads = 576;
 constexpr int kReaders = 512;  // warps 0-15: four warpgroups read TMEM
 constexpr int kProducerWarp = 16;
@@ -389,7 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t c2 = *reinterpret_cast<const uint64_t*>(nc + 2 * e2);  // (-c_r, -c_r+1)
               float t0, t1;
               f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, c2), t0, t1);
-              a2[e2 & 1] = f2_add(a2[e2 & 1], f2_pack(ex2_approx(t0), ex2_approx(t1)));
+              float p0, p1;
+              if (e2 % 3 == 2) {  // one pair in three on the FMA pipe
+                ex2_fma_pair(t0, t1, p0, p1);
+              } else {
+                p0 = ex2_approx(t0);
+                p1 = ex2_approx(t1);
+              }
+              a2[e2 & 1] = f2_add(a2[e2 & 1], f2_pack(p0, p1));
             }
             float s0, s1, s2, s3;
             f2_unpack(a2[0], s0, s1);
@@ -475,6 +528,12 @@ cudaError_t launch_score_tc(const Dims& d, const void* q, const void* k, int win
   const bool two = prm.M > 128;
   if (d.D == 64) return two ? launch_passes<64, 2>(d, mq, mk, prm, st) : launch_passes<64, 1>(d, mq, mk, prm, st);
   return two ? launch_passes<128, 2>(d, mq, mk, prm, st) : launch_passes<128, 1>(d, mq, mk, prm, st);
+}
+
+cudaError_t launch_debug_exp2(const float* x, float* y, int n, cudaStream_t st) {
+  debug_exp2_kernel<<<(n / 2 + 255) / 256, 256, 0, st>>>(x, y, n);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 }  // namespace tsa

@@ -385,6 +385,11 @@ void tsa_debug_set_wait_limit(uint64_t polls) { g_wait_limit.store(polls, std::m
 
 uint64_t tsa_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+tsa_status tsa_debug_exp2(const float* x, float* y, int32_t n, void* stream) {
+  if (!aligned16(x) || !aligned16(y) || n < 2 || (n & 1)) return TSA_ERR_INVALID_ARG;
+  return cuda_status(launch_debug_exp2(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
   uint32_t* base = status_word(ws);
