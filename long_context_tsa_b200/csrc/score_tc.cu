@@ -37,8 +37,8 @@ using namespace tc;
 // ---- 2^t on the FMA pipe, for part of the column-sum exponentials ----
 //
 // The exponential unit (16 results per clock per SM) bounds both passes, so one
-// pair in three of pass 2's exponentials is computed with FMA-pipe arithmetic
-// instead (measured 6 % faster for the score).  Written from the math:
+// pair in three of the exponentials is computed with FMA-pipe arithmetic
+// instead (measured 6 % faster for pass 2).  Written from the math:
 // t = j + f with j = floor(t) and f in [0, 1); 2^f by a degree-4 polynomial
 // p(f) = 1 + f (c1 + f (c2 + f (c3 + f c4))) whose coefficients were fitted to
 // 2^f on [0, 1) by iteratively reweighted least squares on the relative error
@@ -47,7 +47,8 @@ using namespace tc;
 // -infinity, whose low mantissa bits then hold j (the bits of 1.5 * 2^23 shift
 // out of the exponent field).  t is clamped to >= -126 so the result stays a
 // normal float: values below 2^-126 come out as 2^-126 instead of smaller, an
-// absolute error below 1.2e-38 per term.  Valid for t < 128 (pass 2 has t <= 0).
+// absolute error below 1.2e-38 per term.  Valid for t < 128 (pass 2 has t <= 0;
+// pass 1 clamps t to 127 first).
 __device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -332,7 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e2 = 0; e2 < 32; ++e2) {
               float t0, t1;
               f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, negm2), t0, t1);
-              a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(ex2_approx(t0), ex2_approx(t1)));
+              float p0, p1;
+              if (e2 % 3 == 2) {  // one pair in three on the FMA pipe; t <= 127 there (clamped: a
+                                  // larger t saturates at 2^127 and the sum check below redoes the tile)
+                ex2_fma_pair(fminf(t0, 127.f), fminf(t1, 127.f), p0, p1);
+              } else {
+                p0 = ex2_approx(t0);
+                p1 = ex2_approx(t1);
+              }
+              a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(p0, p1));
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
             f2_unpack(a2[0], s0, s1);
