@@ -287,12 +287,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op", default="forward",
-                    choices=["forward", "forward-accumulate", "forward-coverage", "forward-block-sparse", "drift"],
+                    choices=["forward", "forward-accumulate", "forward-coverage", "forward-block-sparse", "drift",
+                             "sweep"],
                     help="forward: score/select/attend (the headline); forward-accumulate: the same with the "
                          "scatter-add attention into a resident output; forward-coverage: budgets chosen per KV "
                          "head from the coverage --tau (one device-to-host copy of the budgets per step); "
                          "forward-block-sparse: attention restricted by a 128 x 128 block mask of --density in the "
-                         "compressed space; drift: the representation-drift pass")
+                         "compressed space; drift: the representation-drift pass; sweep: the sparsity sweep at "
+                         "128K against dense causal attention in the same library (K = L)")
     ap.add_argument("--density", type=float, default=0.5, help="block density for --op forward-block-sparse")
     ap.add_argument("--tau", type=float, default=0.005, help="token coverage for --op forward-coverage")
     args = ap.parse_args()
@@ -306,6 +308,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.op == "drift":
         bench_drift(args, I, world, rank, local)
+        return
+    if args.op == "sweep":
+        bench_sweep(args, I, world, rank, local)
         return
     w = I.WORKLOADS[args.workload]
     budgets = w.budgets(seed=0)
@@ -460,6 +465,78 @@ def main():
         "gpu_launches": launches,
     }
     print(json.dumps(line), flush=True)
+
+
+def bench_sweep(args, I, world, rank, local):
+    """Sparsity sweep at L=131072 against dense causal attention in the same library.
+
+    For each tau in the sweep, K = floor((1 - tau) L) per KV head: the whole step
+    (score, select, attend) and the attention alone are timed; the dense
+    baseline is tsa_attend with K = L (identity permutation), the ordinary causal
+    attention of the layer.  Speedups are dense attention time over the TSA step
+    (what a layer gains, scoring included) and over the TSA attention alone --
+    the quantity the pages quote as "up to 3.23x at 128K" on their own setting."""
+    import long_context_tsa_b200 as T
+
+    if args.impl == "reference" or world > 1:
+        if rank == 0:
+            print(json.dumps({"impl": args.impl, "unavailable": "the sweep is a single-GPU context measurement"}),
+                  flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS["gqa_bf16_L131072"]
+    q, k, v = I.make_qkv(w, seed=0, device=dev)
+    desc = T.desc_for(q, k)
+    ws = T.alloc_workspace(desc, w.W, device=dev)
+    scores = torch.empty((w.B, w.Hkv, w.L), dtype=torch.float32, device=dev)
+    perm = torch.empty((w.B, w.Hkv, w.L), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        for _ in range(max(1, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    dense_b = [w.L] * (w.B * w.Hkv)
+    ident = torch.arange(w.L, dtype=torch.int32, device=dev).expand(w.B, w.Hkv, w.L).contiguous()
+    t_dense = timed(lambda: T.tsa_attend(desc, q, k, v, ident, dense_b, out, ws), 3)
+    rows = []
+    for tau in I.SWEEP_TAUS:
+        budgets = [I.sweep_budget(tau, w.L)] * (w.B * w.Hkv)
+
+        def step():
+            T.tsa_score(desc, q, k, w.W, scores, ws)
+            T.tsa_select(desc, scores, budgets, perm, ws)
+            T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
+
+        t_step = timed(step, args.steps)
+        t_att = timed(lambda: T.tsa_attend(desc, q, k, v, perm, budgets, out, ws), args.steps)
+        fl = attend_flops(w, budgets)
+        rows.append({"tau": tau, "K_per_kv_head": budgets[0], "step_ms": t_step, "attend_ms": t_att,
+                     "attend_tflops": fl / (t_att * 1e-3) / 1e12, "speedup_vs_dense_step": t_dense / t_step,
+                     "speedup_vs_dense_attend": t_dense / t_att})
+    st = T.tsa_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after the sweep: {T.tsa_status_string(st)}")
+    fl_dense = attend_flops(w, dense_b)
+    print(json.dumps({
+        "metric": "attention speedup vs dense causal attention (same library, K = L) at 128K",
+        "unit": "x", "higher_is_better": True, "n_gpus": 1, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "op": "sweep", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D,
+                   "W": w.W},
+        "dense": {"attend_ms": t_dense, "attend_tflops": fl_dense / (t_dense * 1e-3) / 1e12},
+        "sweep": rows,
+        "pages_figure": "up to 3.23x at 128K (hardware and setting not stated on the pages; context only)",
+    }), flush=True)
 
 
 def bench_drift(args, I, world, rank, local):
