@@ -276,3 +276,26 @@ def test_attend_block_sparse_full_mask_equals_attend():
     T.tsa_attend_block_sparse(r.desc, q, k, v, perm_t, budgets, ones, r.out, r.ws)
     assert r.status() == 0
     assert torch.equal(r.out, dense)  # the same kernel path, bit for bit
+
+
+@pytest.mark.parametrize("spike_pos", [700, 1500, 2900])
+def test_score_logit_far_above_the_running_max(spike_pos):
+    # One key whose logit exceeds every earlier key of the window rows by ~200 in
+    # log2 units (q.k = 40 * 40 = 1600, x scale * log2(e) ~ 0.1275): in the row-
+    # statistics pass the tile holding it starts far above the running reference,
+    # the sum leaves the safe range (or saturates at 2^127 in the FMA-pipe lanes)
+    # and the tile is redone against its own maximum.
+    w = I.custom("score_spike", Hq=4, Hkv=1, L=3000, D=128, dtype="bf16", W=32, sigma=0.3)
+    q, k, v = I.make_qkv(w, seed=21, device="cpu")
+    u = torch.randn(128, generator=torch.Generator().manual_seed(22))
+    u = u / u.norm()
+    q = q.float()
+    q[0, :, w.L - w.W:] += 40.0 * u  # every window row points along u
+    k = k.float()
+    k[0, 0, spike_pos] += 40.0 * u
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    r = Run(w, q.to(DEV), k.to(DEV), v.to(DEV))
+    gpu = host(r.score())
+    ora = O.score(host(q), host(k), w.W)
+    assert_scores_close(gpu, ora)
+    assert gpu[0, 0, spike_pos] > 0.99 * w.W * w.G  # the spike takes nearly all of the mass
