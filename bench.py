@@ -283,7 +283,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tsa", choices=["tsa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-slots", type=int, default=2, help="streams / buffer sets the end-to-end leg rotates over")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op", default="forward",
@@ -418,7 +419,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(T, w, desc, q, k, v, budgets, dev, stream, args.e2e_steps, dist)
+        e2e = run_e2e(T, w, desc, q, k, v, budgets, dev, stream, args.e2e_steps, dist, args.e2e_slots)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -625,43 +626,45 @@ def bench_drift(args, I, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist):
+def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist, n_slots=2):
     """Same metric through tsa_forward_host: pinned host inputs copied in, the
     forward, and the full output copied back, all inside the timed region.
 
-    Steps alternate between two streams, each with its own device buffers,
+    Steps rotate over `n_slots` streams, each with its own device buffers,
     workspace and pinned output buffer, the way a server overlaps requests:
-    one step's host-to-device copy runs while the previous step computes and
-    copies its output back (the two directions use separate copy engines)."""
+    one step's host-to-device copy runs while earlier steps compute and copy
+    their outputs back (the two directions use separate copy engines)."""
     qh = q.cpu().pin_memory()
     kh = k.cpu().pin_memory()
     vh = v.cpu().pin_memory()
-    streams = [stream, torch.cuda.Stream(dev)]
+    streams = [stream] + [torch.cuda.Stream(dev) for _ in range(n_slots - 1)]
     slots = []
-    for _ in range(2):
+    for _ in range(n_slots):
         slots.append({"qd": torch.empty_like(q), "kd": torch.empty_like(k), "vd": torch.empty_like(v),
                       "od": torch.empty_like(q), "oh": torch.empty(q.shape, dtype=q.dtype).pin_memory(),
                       "ws": T.alloc_workspace(desc, w.W, device=dev)})
 
     def one(i):
-        sl = slots[i % 2]
+        sl = slots[i % n_slots]
         T.tsa_forward_host(desc, qh, kh, vh, w.W, budgets, sl["oh"], sl["qd"], sl["kd"], sl["vd"], sl["od"],
-                           sl["ws"], stream=streams[i % 2])
+                           sl["ws"], stream=streams[i % n_slots])
 
-    for i in range(2):
+    for i in range(n_slots):
         one(i)
     torch.cuda.synchronize(dev)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     s.record(streams[0])
-    streams[1].wait_event(s)
+    for st_ in streams[1:]:
+        st_.wait_event(s)
     for i in range(steps):
         one(i)
-    e1.record(streams[1])
-    streams[0].wait_event(e1)
+    for st_ in streams[1:]:
+        e1 = torch.cuda.Event()
+        e1.record(st_)
+        streams[0].wait_event(e1)
     e.record(streams[0])
     torch.cuda.synchronize(dev)
     ms = max_over_ranks([s.elapsed_time(e) / steps], dist, dev)[0]
@@ -673,7 +676,7 @@ def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist):
     nb = lambda t: t.numel() * t.element_size()  # noqa: E731
     return {"value": job_tokens_per_s(world, w.B * w.L, ms), "unit": "tokens/s", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
             "d2h_bytes_per_step": nb(q), "ms_per_step": ms, "steps": steps,
-            "pipeline": "two streams, two buffer sets (copies of one step overlap the next)"}
+            "pipeline": f"{n_slots} streams, {n_slots} buffer sets (copies of one step overlap the others)"}
 
 
 def run_reference(args, w, budgets, world):
