@@ -100,10 +100,19 @@ def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: s
     sel_bytes = 2.0 * 4 * w.B * w.Hkv * w.L
     a_sel = sel_bytes / (t_select_ms * 1e-3) / 1e9
     hbm = float(peaks["hbm_gbs"])
+    # score bytes: K read once, the window queries, the scores written (the second pass re-reads K
+    # mostly from L2 and is not counted)
+    esz = 2 if w.dtype == "bf16" else 4
+    sc_bytes = (w.B * w.Hkv * w.L * w.D + w.B * w.Hq * w.W * w.D) * esz + 4.0 * w.B * w.Hkv * w.L
+    a_sc_hbm = sc_bytes / (t_score_ms * 1e-3) / 1e9
     return [
         {"kernel": "score_tc (2 passes)", "bound": "alu", "achieved": a_score / 1e12, "peak": mufu_peak / 1e12,
          "unit": "Tex2/s", "frac": a_score / mufu_peak,
-         "peak_source": f"16 ex2/clk/SM x {sms} SMs x {mhz:.0f} MHz (max SM clock)"},
+         "peak_source": f"16 ex2/clk/SM x {sms} SMs x {mhz:.0f} MHz (max SM clock)",
+         "note": "one exponential pair in three runs on the FMA pipe, so this is an effective rate"},
+        {"kernel": "score_tc (2 passes)", "bound": "hbm", "achieved": a_sc_hbm, "peak": hbm, "unit": "GB/s",
+         "frac": a_sc_hbm / hbm, "peak_source": f"hbm_gbs ({peak_src})",
+         "note": "algorithmic bytes (K once, window queries, scores); the exponentials bound it first"},
         {"kernel": "select_radix", "bound": "hbm", "achieved": a_sel, "peak": hbm, "unit": "GB/s",
          "frac": a_sel / hbm, "peak_source": f"hbm_gbs ({peak_src})", "note": "latency-bound: 64 CTAs, cluster barriers between 4 radix passes"},
     ]

@@ -124,7 +124,7 @@ def compare_attend(out: torch.Tensor, q, k, v, perm_np: np.ndarray, budgets, dty
                 rows = np.arange(K)
             else:
                 pick = rng.choice(K, size=rows_per_head, replace=False)
-                rows = np.unique(np.concatenate([pick, [0, K - 1]]))
+                rows = np.unique(np.concatenate([pick, np.arange(min(4, K)), [K - 1]]))  # first rows hold kept sinks
             ora = O.attend_rows(q, k, v, perm_np[b, g], K, b, h, G, rows)
             pos = torch.from_numpy(perm_np[b, g, rows].astype(np.int64)).to(out.device)
             gpu = host(out[b, h].index_select(0, pos))

@@ -42,7 +42,10 @@ def test_block_mask_for_keeps_diagonal_and_sinks():
 def test_other_rooflines_counts():
     w = I.WORKLOADS["gqa_bf16_L131072"]
     r = bench.other_rooflines(w, 0.19, 0.031, {"hbm_gbs": 6450.3}, "measured")
-    score, select = r
+    score, score_hbm, select = r
+    # K read once, the window queries and the scores written
+    want = (8 * 131072 * 128 + 32 * 64 * 128) * 2 + 4 * 8 * 131072
+    assert abs(score_hbm["achieved"] * 1e9 * 0.19e-3 - want) < 1.0 and score_hbm["bound"] == "hbm"
     # 2 passes x (B x Hkv) groups x (G x W) window rows x L keys exponentials
     assert abs(score["achieved"] * 1e12 * 0.19e-3 - 2 * 8 * 4 * 64 * 131072) < 1e3
     assert score["bound"] == "alu" and 0 < score["frac"] < 1
