@@ -118,6 +118,15 @@ def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: s
     ]
 
 
+def input_checksum(*tensors) -> str:
+    """Sum of the raw element bits of each tensor (int64, on the device): identifies the exact inputs."""
+    parts = []
+    for t in tensors:
+        bits = t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+        parts.append(str(int(bits.to(torch.int64).sum().item())))
+    return ":".join(parts)
+
+
 def rank_seed(rank: int) -> int:
     """Each rank runs its own independent layer (weak scaling): inputs seeded by rank."""
     return rank
@@ -461,7 +470,8 @@ def main():
                    "K_per_kv_head": budgets,
                    "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "
                           f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each; no flush"),
-                   "parallelism": f"{world} independent layers, one per GPU"},
+                   "parallelism": f"{world} independent layers, one per GPU",
+                   "input_checksum": input_checksum(q, k, v)},
         "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend},
         "attend_tflops": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

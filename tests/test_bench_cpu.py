@@ -52,3 +52,14 @@ def test_other_rooflines_counts():
     # scores read once and the permutation written once: 8 bytes per key per group
     assert abs(select["achieved"] * 1e9 * 0.031e-3 - 8 * 8 * 131072) < 1.0
     assert select["bound"] == "hbm" and 0 < select["frac"] < 1
+
+
+def test_input_checksum_depends_on_every_element():
+    import torch
+
+    a = torch.randn(4, 8, generator=torch.Generator().manual_seed(0)).to(torch.bfloat16)
+    b = a.clone()
+    b[3, 7] = -b[3, 7]
+    assert bench.input_checksum(a) == bench.input_checksum(a.clone())
+    assert bench.input_checksum(a) != bench.input_checksum(b)
+    assert len(bench.input_checksum(a, a.float()).split(":")) == 2
