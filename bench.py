@@ -118,6 +118,46 @@ def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: s
     ]
 
 
+def time_zero_dropped(T, w, desc, perm, budgets, out, ws, stream, dev, peaks, peak_src, workload, reps=10):
+    """The scatter's zero rows as a standalone kernel (tsa_zero_dropped) on the step's
+    permutation, against HBM: 2 bytes x D per dropped row per query head written,
+    4 bytes per dropped row read (its position).  In the step itself these zeros are
+    written by spare warps of the attention kernel."""
+    dropped = sum(w.L - min(int(x), w.L) for x in budgets)
+    nbytes = dropped * (w.G * w.D * (2 if w.dtype == "bf16" else 4) + 4)
+    if nbytes == 0:
+        return None
+    for _ in range(3):
+        T.tsa_zero_dropped(desc, perm, budgets, out, ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        T.tsa_zero_dropped(desc, perm, budgets, out, ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    if T.tsa_check_status(ws) != 0:
+        raise RuntimeError("device status after the zero-fill timing")
+    hbm = float(peaks["hbm_gbs"])
+    a = nbytes / (ms * 1e-3) / 1e9
+    traffic, src = kernel_traffic("zero_fill", workload, ["long_context_tsa_b200/csrc/attend_simt.cu"])
+    return {"kernel": "zero_fill (tsa_zero_dropped: the scatter's zero rows, standalone)", "bound": "hbm",
+            "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm, "traffic": traffic,
+            "traffic_source": src, "traffic_capture": capture_note(src), "ms": ms, "algorithmic_bytes": nbytes,
+            "peak_source": f"hbm_gbs ({peak_src})",
+            "note": f"{dropped} dropped rows x {w.G} query heads; timed alone, {reps} launches back to back"}
+
+
+def capture_note(src):
+    """Provenance of a traffic figure read from a committed ncu summary."""
+    if not src:
+        return None
+    text = open(os.path.join(ROOT, src)).read()
+    m = re.search(r"captured:\s*(.+)", text)
+    when = m.group(1).strip() if m else "date not recorded"
+    return f"committed ncu capture {src} ({when}); valid while the kernel source hash matches"
+
+
 def input_checksum(*tensors) -> str:
     """Sum of the raw element bits of each tensor (int64, on the device): identifies the exact inputs."""
     parts = []
@@ -250,45 +290,53 @@ def blas_threads() -> int:
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 
-def oracle_sample(w, q, k, v, budgets, heads, rows_per_head, seed=0):
-    """Time the oracle on a bounded sample and scale it to one full step.
+ORACLE_ROWS_PER_HEAD = 256  # attention rows the oracle computes per query head in one sampled step
 
-    score: `heads` query heads of the window (scaled to all Hq heads);
-    select: the KV groups of those heads (scaled to all B*Hkv groups);
-    attend: `rows_per_head` kept rows of each sampled head (scaled to all kept rows).
-    q, k, v: host float32 arrays.
+
+def oracle_sample(w, q, k, v, budgets, rows_per_head=ORACLE_ROWS_PER_HEAD, seed=0):
+    """Time one sampled step of the oracle and extrapolate it to the full step.
+
+    The one sampling scheme of both CPU legs (the GPU line's cpu_baseline and
+    --impl reference): score over every query head (full), select over every KV
+    group (full), attention on `rows_per_head` seeded kept rows of every query
+    head, the attention time scaled by (all kept rows) / (sampled rows).
+    q, k, v: host float32 arrays.  Returns a dict with the measured wall time,
+    the per-part times, the scale factor and the extrapolated full-step time.
     """
     from oracle import tsa_oracle as O
 
     rng = np.random.default_rng(seed)
-    hs = sorted(rng.choice(w.Hq, size=min(heads, w.Hq), replace=False).tolist())
-    groups = sorted({h // w.G for h in hs})
     t0 = time.perf_counter()
-    sc = {}
-    for h in hs:
-        g = h // w.G
-        part = O.score(q[:, h:h + 1], k[:, g:g + 1], w.W)
-        sc[g] = sc.get(g, 0.0) + part[0, 0]
+    sc = O.score(q, k, w.W)
     t1 = time.perf_counter()
-    perms = {}
-    for g in groups:
-        perms[g] = O.select(np.asarray(sc[g], dtype=np.float32)[None, None, :], [budgets[g]])[0, 0]
+    perm = O.select(sc.astype(np.float32), budgets)
     t2 = time.perf_counter()
+    kept = O.clamp_budgets(budgets, w.L)
     n_rows = 0
-    for h in hs:
-        g = h // w.G
-        K = min(budgets[g], w.L)
-        rows = rng.choice(K, size=min(rows_per_head, K), replace=False)
-        O.attend_rows(q, k, v, perms[g], K, 0, h, w.G, rows)
-        n_rows += rows.size
+    for b in range(w.B):
+        for h in range(w.Hq):
+            g = h // w.G
+            K = int(kept[b * w.Hkv + g])
+            rows = rng.choice(K, size=min(rows_per_head, K), replace=False)
+            O.attend_rows(q, k, v, perm[b, g], K, b, h, w.G, rows)
+            n_rows += rows.size
     t3 = time.perf_counter()
-    total_rows = sum(w.G * min(budgets[g], w.L) for g in range(w.B * w.Hkv))
-    est = (t1 - t0) * (w.B * w.Hq / len(hs)) + (t2 - t1) * (w.B * w.Hkv / len(groups)) + \
-        (t3 - t2) * (total_rows / max(1, n_rows))
-    sample = (f"score {len(hs)}/{w.B * w.Hq} query heads (x{w.B * w.Hq / len(hs):.0f}), select "
-              f"{len(groups)}/{w.B * w.Hkv} KV groups (x{w.B * w.Hkv / len(groups):.0f}), attend {n_rows} of "
-              f"{total_rows} kept rows (x{total_rows / max(1, n_rows):.1f}); fp64 numpy")
-    return est, t3 - t0, sample
+    total_rows = int(sum(w.G * int(x) for x in kept))
+    scale = total_rows / max(1, n_rows)
+    est = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale
+    sample = (f"score all {w.B * w.Hq} query heads and select all {w.B * w.Hkv} KV groups in full; attention on "
+              f"{rows_per_head} seeded kept rows per query head ({n_rows} of {total_rows} kept rows, time scaled "
+              f"x{scale:.1f}); fp64 numpy")
+    return {"wall_s": t3 - t0, "score_s": t1 - t0, "select_s": t2 - t1, "attend_s": t3 - t2, "attend_scale": scale,
+            "est_s": est, "sample": sample}
+
+
+def make_inputs(I, w, seed):
+    """The workload's seeded inputs, drawn by torch's CUDA generator when a GPU is
+    present (both arms then time the same tensors), else by its CPU generator."""
+    if torch.cuda.is_available():
+        return I.make_qkv(w, seed=seed, device="cuda"), "torch CUDA generator"
+    return I.make_qkv(w, seed=seed, device="cpu"), "torch CPU generator (no GPU on this host)"
 
 
 # ----------------------------------------------------------------------------- main
@@ -350,7 +398,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
 
-    q, k, v = I.make_qkv(w, seed=rank_seed(rank), device=dev)
+    q, k, v = I.make_qkv(w, seed=rank_seed(rank), device=dev)  # the reference arm draws the same tensors
     desc = T.desc_for(q, k)
     ws = T.alloc_workspace(desc, w.W, device=dev)
     scores = torch.empty((w.B, w.Hkv, w.L), dtype=torch.float32, device=dev)
@@ -396,6 +444,9 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {T.tsa_status_string(st)}")
 
+    # L2 (126 MB) is flushed between timed steps by writing a 256 MB buffer; each step
+    # is timed by its own events, so the flushes sit outside the step times.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -408,6 +459,7 @@ def main():
     launches0 = T.tsa_debug_launch_count()
     start.record(stream)
     for i in range(args.steps):
+        flush.zero_()
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -419,12 +471,13 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status after timing: {T.tsa_status_string(st)}")
 
-    total_ms = start.elapsed_time(end)
+    loop_ms = start.elapsed_time(end)  # includes the flushes
+    steps_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
     t_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     t_attend = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms, t_attend = max_over_ranks([total_ms, t_attend], dist, dev)
-    ms_per_step = total_ms / args.steps
+    steps_ms, t_attend, loop_ms = max_over_ranks([steps_ms, t_attend, loop_ms], dist, dev)
+    ms_per_step = steps_ms / args.steps
     tokens = w.B * w.L
     value = job_tokens_per_s(world, tokens, ms_per_step)
 
@@ -434,6 +487,9 @@ def main():
     peak = float(peaks["bf16_tflops"])
     traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
                                                                        "long_context_tsa_b200/csrc/tc_ptx.cuh"])
+    zf = None
+    if not coverage:
+        zf = time_zero_dropped(T, w, desc, perm, budgets, out, ws, stream, dev, peaks, peak_src, args.workload)
 
     e2e = None
     if not args.no_e2e:
@@ -442,9 +498,12 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         qn, kn, vn = (t.float().cpu().numpy() for t in (q, k, v))
-        est, wall, sample = oracle_sample(w, qn, kn, vn, budgets, heads=w.Hq, rows_per_head=256)
-        cpu = {"value": tokens / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": sample + f"; {wall:.1f} s of CPU work, estimated full step {est:.1f} s"}
+        res = oracle_sample(w, qn, kn, vn, budgets)
+        cpu = {"value": tokens / res["est_s"], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": res["sample"] + f"; {res['wall_s']:.1f} s of CPU work, extrapolated full step "
+                                         f"{res['est_s']:.1f} s",
+               "measured_wall_ms_per_step": res["wall_s"] * 1e3, "full_step_ms_estimated": res["est_s"] * 1e3,
+               "attend_scale": res["attend_scale"]}
 
     if dist is not None:
         dist.barrier()
@@ -468,8 +527,10 @@ def main():
                    "block_density": args.density if block_sparse else None,
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets,
-                   "l2": (f"inputs larger than L2 (126 MB): q {q.numel() * q.element_size() / 1e9:.2f} GB, "
-                          f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each; no flush"),
+                   "l2": ("flushed between timed steps (a 256 MB buffer written outside the per-step events); "
+                          f"inputs also exceed L2: q {q.numel() * q.element_size() / 1e9:.2f} GB, "
+                          f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each"),
+                   "timed_loop_ms_incl_flushes": loop_ms,
                    "parallelism": f"{world} independent layers, one per GPU",
                    "input_checksum": input_checksum(q, k, v)},
         "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend},
@@ -477,8 +538,8 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"bf16_tflops ({peak_src})",
                      "kernel": "attend_tc (tsa_attend: gather + attention + scatter + zero fill)",
-                     "traffic_source": traffic_src},
-        "rooflines_other": other_rooflines(w, t_score, t_select, peaks, peak_src),
+                     "traffic_source": traffic_src, "traffic_capture": capture_note(traffic_src)},
+        "rooflines_other": other_rooflines(w, t_score, t_select, peaks, peak_src) + ([zf] if zf else []),
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
@@ -699,20 +760,31 @@ def run_e2e(T, w, desc, q, k, v, budgets, dev, stream, steps, dist, n_slots=2):
 
 
 def run_reference(args, w, budgets, world):
-    """The oracle arm: W warm-up and K timed steps, each a bounded sample of the
-    workload scaled to one full step, on the host cores (rank 0 only)."""
+    """The oracle arm: W warm-up and K timed steps on the host cores (rank 0 only).
+
+    Each step is one sampled oracle step (``oracle_sample``): `ms_per_step` is the
+    wall time those steps actually took; `value` extrapolates each to the full
+    layer (score and select in full, attention rows scaled) and reports tokens/s
+    of the full step."""
     from long_context_tsa_b200 import inputs as I
 
-    q, k, v = I.make_qkv(w, seed=0, device="cpu")
-    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
-    ests = []
-    sample = ""
+    (q, k, v), gen = make_inputs(I, w, seed=0)
+    checksum = input_checksum(q, k, v)
+    qn, kn, vn = (t.float().cpu().numpy() for t in (q, k, v))
+    del q, k, v
+    walls, ests = [], []
+    res = None
     for i in range(args.warmup + args.steps):
-        est, wall, sample = oracle_sample(w, qn, kn, vn, budgets, heads=1, rows_per_head=256, seed=i)
+        res = oracle_sample(w, qn, kn, vn, budgets, seed=i)
         if i >= args.warmup:
-            ests.append(est)
-    ms = statistics.mean(ests) * 1e3
-    value = w.B * w.L / (ms / 1e3)
+            walls.append(res["wall_s"])
+            ests.append(res["est_s"])
+    ms = statistics.mean(walls) * 1e3
+    est_ms = statistics.mean(ests) * 1e3
+    value = w.B * w.L / (est_ms / 1e3)
+    cpu = {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": res["sample"] + " per step",
+           "measured_wall_ms_per_step": ms, "full_step_ms_estimated": est_ms, "attend_scale": res["attend_scale"]}
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -727,10 +799,14 @@ def run_reference(args, w, budgets, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "op": args.op, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
-                   "K_per_kv_head": budgets},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample + " per step"},
+        "config": {"workload": args.workload, "op": args.op, "tau": None, "block_density": None,
+                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
+                   "K_per_kv_head": budgets, "parallelism": "rank 0 only, host cores",
+                   "input_checksum": checksum, "inputs": gen},
+        "timing": (f"ms_per_step is the measured wall time of one sampled oracle step ({ms:.0f} ms); value is "
+                   f"B*L over the full step extrapolated from it ({est_ms:.0f} ms: score and select measured in "
+                   f"full, attention x{res['attend_scale']:.1f})"),
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

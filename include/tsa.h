@@ -128,19 +128,36 @@ TSA_API tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k
                       size_t ws_bytes, void* stream);
 
 /*
+ * tsa_zero_dropped -- the zero rows of the scatter on their own ([P1] Step 2
+ * scatter_attention_output builds the full-length output from zeros; [P2]
+ * Figure 3 scatters into the full sequence layout): for each (b, g) with
+ * K = min(budget_host[b*Hkv+g], L), out[b, h, p, :] = +0 for every dropped
+ * position p in perm[b,g,K:L] and every query head h of group g.  Kept rows
+ * are not touched.  tsa_attend writes these zeros itself; this call is the
+ * same step as one standalone kernel (for callers that write the kept rows
+ * another way, and to measure the step).  Same pointer, budget and
+ * permutation rules as tsa_attend.
+ */
+TSA_API tsa_status tsa_zero_dropped(const tsa_desc* desc, const int32_t* perm, const int32_t* budget_host,
+                                    void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * tsa_score_noalloc -- tsa_score without a caller workspace, for callers that
  * cannot allocate device memory (for example a plugin inside an engine that
  * owns all device memory, or a latency-critical loop that must not call
  * cudaMalloc).  The pages have no counterpart: this is a deployment variant.
- * Same arguments, layout and result as tsa_score; the per-split partials go
- * to a fixed 1 MiB array built into the library, reserved on every GPU that
- * loads it until the process exits.  A shape whose partials exceed 1 MiB
- * (B*Hkv * splits * G*window rounded up to 64 * 8 bytes, splits =
- * ceil(296 / (B*Hkv)) capped by ceil(L/64)) returns TSA_ERR_WORKSPACE; the
- * 32/8-head, window-64 layer fits up to B = 64.  The first call made with a device current looks up the
- * array's device address; make that first call before any stream capture.
- * All calls share the array: calls whose kernels overlap on the GPU race and
- * give wrong scores, so order them on one stream.  Allocates nothing.
+ * Same arguments, layout, kernels and result as tsa_score (tensor-core passes
+ * for bf16, SIMT passes for f32); the per-split partials go to a fixed 1 MiB
+ * array built into the library, reserved on every GPU that loads it until the
+ * process exits.  Checks run in this order: the shape (as tsa_score), then
+ * the partials' size -- B*Hkv * splits * padded window rows * 8 bytes above
+ * 1 MiB returns TSA_ERR_WORKSPACE (the 32/8-head, window-64 layer fits up to
+ * B = 64) -- then the pointers (TSA_ERR_INVALID_ARG).  The first call made
+ * with a device current looks up the array's device address; make that first
+ * call before any stream capture.  All calls share the array: calls whose
+ * kernels overlap on the GPU race and give wrong scores, so order them on one
+ * stream.  Device-side errors go to a status word of the library, read (and
+ * cleared) by tsa_check_status(NULL, 0, stream).  Allocates nothing.
  */
 TSA_API tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const void* k, int32_t window,
                                      float* scores, void* stream);
@@ -259,7 +276,8 @@ TSA_API tsa_status tsa_layer_stable(const double* history, int32_t n, int32_t wi
                                     int32_t* stable);
 
 /* Synchronise `stream`, return the device status recorded in `ws` (TSA_OK,
- * TSA_ERR_TIMEOUT or TSA_ERR_DEVICE_BOUNDS) and clear it. */
+ * TSA_ERR_TIMEOUT or TSA_ERR_DEVICE_BOUNDS) and clear it.  ws = NULL reads
+ * the status word of tsa_score_noalloc on the current device instead. */
 TSA_API tsa_status tsa_check_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Static description of a status code. */

@@ -30,9 +30,11 @@ from ._native import (  # noqa: F401
     tsa_forward_host,
     tsa_layer_stable,
     tsa_score,
+    tsa_score_noalloc,
     tsa_select,
     tsa_select_coverage,
     tsa_status_string,
     tsa_workspace_init,
     tsa_workspace_size,
+    tsa_zero_dropped,
 )

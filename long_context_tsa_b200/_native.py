@@ -24,7 +24,7 @@ EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
-            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2")
+            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2", "tsa_zero_dropped")
 
 
 class TsaDesc(ctypes.Structure):
@@ -59,6 +59,7 @@ _SIGS = {
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_zero_dropped": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _SZ, _P]),
     "tsa_debug_exp2": (ctypes.c_int, [_P, _P, _I32, _P]),
     "tsa_attend_block_sparse": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_select_coverage": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, ctypes.c_double, _P, _P, _P, _SZ, _P]),
@@ -150,6 +151,12 @@ def tsa_attend(desc, q, k, v, perm, budgets, out, ws, stream=None):
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "tsa_attend")
 
 
+def tsa_zero_dropped(desc, perm, budgets, out, ws, stream=None):
+    """+0 at every dropped row of every query head; kept rows untouched."""
+    _check(lib().tsa_zero_dropped(ctypes.byref(desc), _ptr(perm), _budgets(budgets), _ptr(out), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "tsa_zero_dropped")
+
+
 def tsa_attend_accumulate(desc, q, k, v, perm, budgets, out, ws, stream=None):
     """out[kept rows] += attention (scatter-add); dropped rows are left as they are."""
     _check(lib().tsa_attend_accumulate(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
@@ -170,8 +177,16 @@ def tsa_forward_host(desc, q_host, k_host, v_host, window, budgets, out_host, q_
 
 
 def tsa_check_status(ws, stream=None) -> int:
-    """Synchronise, return the device status code recorded in ``ws`` (0 = ok) and clear it."""
-    return int(lib().tsa_check_status(_ptr(ws), ws.numel(), _stream(stream)))
+    """Synchronise, return the device status code recorded in ``ws`` (0 = ok) and clear it.
+
+    ``ws=None`` reads the status word of ``tsa_score_noalloc`` on the current device."""
+    return int(lib().tsa_check_status(_ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def tsa_score_noalloc(desc, q, k, window, scores, stream=None):
+    """tsa_score with the library's fixed scratch instead of a caller workspace."""
+    _check(lib().tsa_score_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), int(window), _ptr(scores),
+                                   _stream(stream)), "tsa_score_noalloc")
 
 
 def tsa_status_string(code: int) -> str:

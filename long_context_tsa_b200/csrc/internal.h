@@ -31,6 +31,15 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const Dims& d, int window);
+
+// Argument checks shared by the entry points (same status codes everywhere).
+bool aligned16(const void* p);
+tsa_status check_desc(const tsa_desc* desc, Dims* d);  // fills d on TSA_OK
+tsa_status check_window(const Dims& d, int window);
+// Bytes of per-split score partials the score passes of d.dtype need.
+size_t score_partials_bytes(const Dims& d, int window);
+// Device address of tsa_score_noalloc's status word on the current device.
+cudaError_t noalloc_status_word(uint32_t** word);
 int score_splits(const Dims& d);
 int window_rows_padded(const Dims& d, int window);  // Mp: G*window rounded up to 64
 

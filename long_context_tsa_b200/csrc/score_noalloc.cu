@@ -8,14 +8,18 @@
 // imply) is not acceptable, or a deployment with a fixed memory budget that
 // must not fail with out-of-memory part-way through a run.  This variant keeps
 // the scratch in a fixed array that is part of the library itself, so the
-// caller passes only the inputs and the output.
+// caller passes only the inputs and the output.  It runs the same kernels as
+// tsa_score (tensor-core passes for bf16, SIMT passes for f32), so its scores
+// are those of tsa_score.
 //
 // The array below is reserved on every GPU that loads this library and stays
 // there until the process exits.  It is shared by all calls: two calls whose
 // kernels overlap on the GPU (different streams, or different host threads)
 // overwrite each other's partials and produce wrong scores.  The partials are
 // written in full by the first pass before the second pass reads them, so no
-// part of the array has to start at zero.
+// part of the array has to start at zero.  The device status word (a bounded
+// wait that ran out) is cleared by each call and read back by
+// tsa_check_status(NULL, 0, stream).
 #include <math.h>
 
 #include <mutex>
@@ -27,8 +31,8 @@ namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t{1} << 20;  // 1 MiB of partials
 
-// Host code sees this name only as a stand-in: its device address comes from
-// cudaGetSymbolAddress, once per device.
+// Host code sees these names only as stand-ins: their device addresses come
+// from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) float g_score_scratch[kNoAllocScratchBytes / sizeof(float)];
 static __device__ __align__(256) uint32_t g_score_status[64];
 
@@ -37,9 +41,9 @@ std::mutex g_mu;
 float* g_scratch_ptr[kMaxDevices] = {};
 uint32_t* g_status_ptr[kMaxDevices] = {};
 
-// Device address of the fixed scratch on the current device (looked up on the
-// first call made with that device current).
-cudaError_t scratch_for_current_device(float** scratch, uint32_t** status) {
+// Device addresses of the fixed scratch and status word on the current device
+// (looked up on the first call made with that device current).
+cudaError_t fixed_buffers_for_current_device(float** scratch, uint32_t** status) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -60,37 +64,33 @@ cudaError_t scratch_for_current_device(float** scratch, uint32_t** status) {
   return cudaSuccess;
 }
 
-bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
+
+cudaError_t noalloc_status_word(uint32_t** word) {
+  float* scratch = nullptr;
+  return fixed_buffers_for_current_device(&scratch, word);
+}
+
 }  // namespace tsa
 
 using namespace tsa;
 
 extern "C" tsa_status tsa_score_noalloc(const tsa_desc* desc, const void* q, const void* k, int32_t window,
                                         float* scores, void* stream) {
-  if (desc == nullptr) return TSA_ERR_INVALID_ARG;
-  // Same shape rules as tsa_score (the workspace size is the probe: 0 = invalid).
-  if (tsa_workspace_size(desc, window) == 0) {
-    if (desc->D != 64 && desc->D != 128) return TSA_ERR_UNSUPPORTED;
-    return TSA_ERR_INVALID_ARG;
-  }
-  if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return TSA_ERR_INVALID_ARG;
+  // Shape first, then the fixed scratch's size limit, then the pointers: a shape
+  // the array cannot hold is refused before any pointer is looked at.
   Dims d;
-  d.B = desc->B;
-  d.Hq = desc->Hq;
-  d.Hkv = desc->Hkv;
-  d.L = desc->L;
-  d.D = desc->D;
-  d.G = desc->Hq / desc->Hkv;
-  d.dtype = desc->dtype;
-  d.scale = desc->scale > 0.f ? desc->scale : 1.0f / sqrtf((float)desc->D);
-  const size_t need = (size_t)d.B * d.Hkv * score_splits(d) * window_rows_padded(d, window) * 2 * sizeof(float);
-  if (need > kNoAllocScratchBytes) return TSA_ERR_WORKSPACE;  // shape needs more than the fixed 1 MiB
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if ((s = check_window(d, window)) != TSA_OK) return s;
+  if (score_partials_bytes(d, window) > kNoAllocScratchBytes) return TSA_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return TSA_ERR_INVALID_ARG;
   float* scratch = nullptr;
   uint32_t* status = nullptr;
-  if (scratch_for_current_device(&scratch, &status) != cudaSuccess) return TSA_ERR_CUDA;
+  if (fixed_buffers_for_current_device(&scratch, &status) != cudaSuccess) return TSA_ERR_CUDA;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
-  return launch_score_simt(d, q, k, window, scores, scratch, status, st) == cudaSuccess ? TSA_OK : TSA_ERR_CUDA;
+  const cudaError_t e = d.dtype == TSA_BF16 ? launch_score_tc(d, q, k, window, scores, scratch, status, st)
+                                            : launch_score_simt(d, q, k, window, scores, scratch, status, st);
+  return e == cudaSuccess ? TSA_OK : TSA_ERR_CUDA;
 }

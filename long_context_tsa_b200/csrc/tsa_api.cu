@@ -60,9 +60,14 @@ WsLayout ws_layout(const Dims& d, int window) {
   return w;
 }
 
-namespace {
-
-constexpr size_t kHeaderBytes = 256;
+size_t score_partials_bytes(const Dims& d, int window) {
+  const size_t groups = (size_t)d.B * d.Hkv;
+  if (d.dtype == TSA_BF16) {  // tensor-core passes: window rows padded to 128 or 256
+    const size_t Mp_tc = d.G * window > 128 ? 256 : 128;
+    return groups * (size_t)score_tc_splits(d) * Mp_tc * 2 * sizeof(float);
+  }
+  return groups * (size_t)score_splits(d) * (size_t)window_rows_padded(d, window) * 2 * sizeof(float);
+}
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -93,6 +98,10 @@ tsa_status check_window(const Dims& d, int window) {
   if (d.G * window > kMaxWindowRows) return TSA_ERR_UNSUPPORTED;
   return TSA_OK;
 }
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
 
 tsa_status load_budgets(const Dims& d, const int32_t* budget_host, Budgets* kb) {
   if (budget_host == nullptr) return TSA_ERR_INVALID_ARG;
@@ -216,6 +225,18 @@ tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const 
   Budgets kb;
   if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
   return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_zero_dropped(const tsa_desc* desc, const int32_t* perm, const int32_t* budget_host, void* out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (!aligned16(perm) || !aligned16(out) || !aligned16(ws)) return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return cuda_status(launch_zero_fill(d, perm, kb, out, status_word(ws), static_cast<cudaStream_t>(stream)));
 }
 
 tsa_status tsa_attend_accumulate(const tsa_desc* desc, const void* q, const void* k, const void* v,
@@ -351,12 +372,18 @@ tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void
 }
 
 tsa_status tsa_check_status(void* ws, size_t ws_bytes, void* stream) {
-  if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
+  uint32_t* word_dev = nullptr;
+  if (ws == nullptr) {  // the status word of tsa_score_noalloc on the current device
+    if (noalloc_status_word(&word_dev) != cudaSuccess) return TSA_ERR_CUDA;
+  } else {
+    if (!aligned16(ws) || ws_bytes < kHeaderBytes) return TSA_ERR_INVALID_ARG;
+    word_dev = status_word(ws);
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return TSA_ERR_CUDA;
   uint32_t word = 0;
-  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return TSA_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaMemcpy(&word, word_dev, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaMemsetAsync(word_dev, 0, sizeof(word), st) != cudaSuccess) return TSA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return TSA_ERR_CUDA;
   switch (word) {
     case TSA_OK:

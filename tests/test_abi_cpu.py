@@ -142,6 +142,29 @@ def test_next_row_calls_reject_before_launch(lib):
                                     256, None) == wsz
 
 
+def test_zero_dropped_and_noalloc_reject_before_launch(lib):
+    d = desc()
+    b = N._budgets([4096] * 8)
+    bad_b = N._budgets([4096] * 7 + [-1])
+    inv, wsz = N.STATUS["TSA_ERR_INVALID_ARG"], N.STATUS["TSA_ERR_WORKSPACE"]
+    assert lib.tsa_zero_dropped(ctypes.byref(d), FAKE, bad_b, FAKE, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_zero_dropped(ctypes.byref(d), FAKE + 4, b, FAKE, FAKE, 1 << 20, None) == inv
+    assert lib.tsa_zero_dropped(ctypes.byref(d), FAKE, b, FAKE, FAKE, 16, None) == wsz
+    assert lib.tsa_zero_dropped(ctypes.byref(desc(D=96)), FAKE, b, FAKE, FAKE, 1 << 20, None) == \
+        N.STATUS["TSA_ERR_UNSUPPORTED"]
+    # The no-allocation scorer checks the shape, then its fixed scratch, then the pointers:
+    # B = 65 with 32/8 heads and window 64 needs more than its 1 MiB, whatever the pointers.
+    for dt in (N.TSA_BF16, N.TSA_F32):
+        big = N.make_desc(B=65, Hq=32, Hkv=8, L=8192, D=128, dtype=dt)
+        assert lib.tsa_score_noalloc(ctypes.byref(big), None, None, 64, None, None) == wsz
+        fits = N.make_desc(B=64, Hq=32, Hkv=8, L=256, D=128, dtype=dt)
+        assert lib.tsa_score_noalloc(ctypes.byref(fits), None, None, 64, None, None) == inv
+    assert lib.tsa_score_noalloc(ctypes.byref(desc(D=96)), None, None, 64, None, None) == \
+        N.STATUS["TSA_ERR_UNSUPPORTED"]
+    assert lib.tsa_score_noalloc(ctypes.byref(desc()), None, None, 65, None, None) == \
+        N.STATUS["TSA_ERR_UNSUPPORTED"]  # G * W = 260 > 256, the same code tsa_score returns
+
+
 def test_binding_checks_block_mask_shape():
     import torch
 

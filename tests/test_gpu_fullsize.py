@@ -19,7 +19,7 @@ from .parity_util import Run, assert_dropped_rows_zero, assert_rows_close, asser
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-ROWS = 128  # sampled kept rows per query head (plus the first four: sinks, when kept, sit there)
+ROWS = 512  # sampled kept rows per query head (plus the first four -- kept sinks sit there -- and the last)
 
 
 def _setup(name, seed=0):
@@ -60,7 +60,7 @@ def test_ragged_budgets_and_sparsity_sweep_131072():
         perm = O.select(s32, budgets)
         np.testing.assert_array_equal(host(r.select(torch.from_numpy(s32).to(DEV), budgets)), perm)
         out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
-        compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=16, seed=2)
+        compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=ROWS, seed=2)
         assert_dropped_rows_zero(out, torch.from_numpy(perm).to(DEV), budgets, w.G)
 
 
@@ -71,7 +71,7 @@ def test_dense_keep_all_131072():
     perm = np.broadcast_to(np.arange(w.L, dtype=np.int64), (w.B, w.Hkv, w.L)).copy()
     r = Run(w, q, k, v)
     out = r.attend(torch.from_numpy(perm.astype(np.int32)).to(DEV), budgets)
-    compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=8, seed=3)
+    compare_attend(out, qn, kn, vn, perm, budgets, w.dtype, rows_per_head=ROWS, seed=3)
 
 
 def test_block_sparse_131072():
@@ -92,10 +92,10 @@ def test_block_sparse_131072():
     assert r.status() == 0
     kept = O.clamp_budgets(budgets, w.L)
     rs = np.random.default_rng(6)
-    for h in range(0, w.Hq, 3):
+    for h in range(w.Hq):
         g = h // w.G
         K = int(kept[g])
-        rows = np.unique(np.concatenate([rs.choice(K, 24, replace=False), [0, K - 1]]))
+        rows = np.unique(np.concatenate([rs.choice(K, ROWS, replace=False), np.arange(4), [K - 1]]))
         ora = O.attend_rows(qn, kn, vn, perm[0, g], K, 0, h, w.G, rows, block_mask_bg=bm[0, g])
         pos = torch.from_numpy(perm[0, g, rows]).to(DEV)
         assert_rows_close(host(r.out[0, h].index_select(0, pos)), ora, w.dtype, f"h={h}")
@@ -119,9 +119,32 @@ def test_accumulate_8192_many_items_per_cta():
     for h in range(w.Hq):
         g = h // w.G
         K = int(kept[g])
-        rows = np.unique(np.concatenate([rs.choice(K, 32, replace=False), [0, K - 1]]))
+        rows = np.unique(np.concatenate([rs.choice(K, ROWS, replace=False), np.arange(4), [K - 1]]))
         ora = bn[0, h, perm[0, g, rows]] + O.attend_rows(qn, kn, vn, perm[0, g], K, 0, h, w.G, rows)
         pos = torch.from_numpy(perm[0, g, rows]).to(DEV)
         assert_rows_close(host(out[0, h].index_select(0, pos)), ora, w.dtype, f"h={h}")
         drop = torch.from_numpy(perm[0, g, K:]).to(DEV)
         assert torch.equal(out[0, h].index_select(0, drop), base[0, h].index_select(0, drop))
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32_L256", "gqa_bf16_L131072", "ragged_bf16_L131072"])
+def test_zero_dropped_standalone(name):
+    # The scatter's zero rows on their own: +0 at every dropped row of every query
+    # head, kept rows left exactly as they were.
+    w = I.WORKLOADS[name]
+    q, k, _ = I.make_qkv(w, seed=0, device=DEV)
+    budgets = w.budgets(seed=1)
+    perm = O.select(np.random.default_rng(11).random((w.B, w.Hkv, w.L)).astype(np.float32), budgets)
+    perm_d = torch.from_numpy(perm.astype(np.int32)).to(DEV)
+    base = torch.randn(q.shape, generator=torch.Generator(device=DEV).manual_seed(12), device=DEV).to(q.dtype)
+    out = base.clone()
+    desc = T.desc_for(q, k)
+    ws = T.alloc_workspace(desc, w.W, device=DEV)
+    T.tsa_zero_dropped(desc, perm_d, budgets, out, ws)
+    assert T.tsa_check_status(ws) == 0
+    assert_dropped_rows_zero(out, perm_d, budgets, w.G)
+    kept = O.clamp_budgets(budgets, w.L)
+    for g in range(w.Hkv):
+        keep = torch.from_numpy(perm[0, g, :int(kept[g])]).to(DEV)
+        hs = slice(g * w.G, (g + 1) * w.G)
+        assert torch.equal(out[0, hs].index_select(1, keep), base[0, hs].index_select(1, keep))

@@ -522,3 +522,111 @@ def test_block_sparse_full_mask_is_attend_and_diagonal_mask_is_blockwise():
             ref = O.attend(q[:, hs][:, :, sub[0, 0]], k[:, g:g + 1][:, :, sub[0, 0]], v[:, g:g + 1][:, :, sub[0, 0]],
                            sub_perm, [n])
             np.testing.assert_allclose(out[0, hs][:, sub[0, 0]], ref[0], rtol=0, atol=1e-12)
+
+
+# --- fixed-point token masses: hand values and exact integer bounds --------------------------
+#
+# The coverage reading makes a token's mass the integer floor(clamp(s, 0, 256) * 2^S) with
+# S = 55 - ceil(log2 L): the largest shift for which L tokens of the largest score (256) still sum
+# to at most 2^63 in a 64-bit integer.  These pins do not call the oracle's formula back: they
+# state hand-computed masses and check the bound with exact Python integers, so a shift off by one
+# in either direction fails them (see the mutation test below).
+
+
+def _mass(x, L):
+    return int(O.token_mass(np.array([x], dtype=np.float32), L)[0])
+
+
+def _pin_coverage_masses():
+    L = 131072  # 2^17, so the shift is 55 - 17 = 38
+    assert _mass(256.0, L) == 2 ** 46  # 2^8 * 2^38
+    assert _mass(1.0e6, L) == 2 ** 46  # clamped at 256 first
+    assert _mass(1.0, L) == 2 ** 38
+    assert _mass(2.0 ** -38, L) == 1  # the smallest score that weighs anything
+    assert _mass(2.0 ** -39, L) == 0
+    assert _mass(3 * 2.0 ** -38, L) == 3
+    assert _mass(1.5 * 2.0 ** -38, L) == 1  # floor, not round
+    assert _mass(np.float32(1e-45), L) == 0  # a subnormal weighs nothing
+    assert _mass(-3.0, L) == 0 and _mass(np.nan, L) == 0  # negative scores and NaN weigh nothing
+    # A float32 value that is not a dyadic fraction of short length: floor of its exact product.
+    from fractions import Fraction
+
+    x = np.float32(0.1)
+    assert _mass(x, L) == math.floor(Fraction(float(x)) * 2 ** 38)
+    # Shifts by hand at small lengths: ceil(log2 L) = 0, 1, 2, 2, 3.
+    assert _mass(256.0, 1) == 2 ** 63
+    assert _mass(1.0, 2) == 2 ** 54
+    assert _mass(1.0, 3) == 2 ** 53
+    assert _mass(1.0, 4) == 2 ** 53
+    assert _mass(1.0, 5) == 2 ** 52
+
+
+def _pin_coverage_total_bound():
+    lengths = [1, 2, 3, 4, 5, 7, 8, 9, 1000, 8192, 131071, 131072, 131073, 2 ** 30, 2 ** 30 + 1, 2 ** 31 - 1]
+    for L in lengths:
+        top = _mass(256.0, L)  # the most a single token can weigh at this length
+        assert L * top <= 2 ** 63, L  # a head of L such tokens fits the 64-bit total ...
+        assert 2 * L * top > 2 ** 63, L  # ... and one more bit of precision would not
+    # The largest supported length: an all-256 head stays strictly below 2^63.
+    L = 2 ** 31 - 1
+    assert L * _mass(256.0, L) == (2 ** 31 - 1) * 2 ** 32 < 2 ** 63
+
+
+def test_coverage_token_mass_hand_values():
+    _pin_coverage_masses()
+
+
+def test_coverage_head_total_fits_64_bits_and_shift_is_largest():
+    _pin_coverage_total_bound()
+
+
+@pytest.mark.filterwarnings("ignore:invalid value encountered in cast")  # 2^64 overflows the uint64 cast
+@pytest.mark.parametrize("delta", [-1, 1])
+def test_coverage_mass_pins_catch_a_shift_off_by_one(monkeypatch, delta):
+    true_shift = O.coverage_shift
+    monkeypatch.setattr(O, "coverage_shift", lambda L: true_shift(L) + delta)
+    with pytest.raises(AssertionError):
+        _pin_coverage_masses()
+    with pytest.raises(AssertionError):
+        _pin_coverage_total_bound()
+
+
+# --- the composed forward against an independent construction -------------------------------
+
+
+def test_forward_matches_independent_construction():
+    # Score by plain loops (Step 1 written out element by element), the kept set by
+    # enumerating every K-subset, and the attention by PyTorch SDPA with the mask
+    # "kept and causal" written out at full length; dropped rows are zero.
+    r = np.random.default_rng(77)
+    B, Hq, Hkv, L, D, W = 1, 4, 2, 10, 4, 3
+    G = Hq // Hkv
+    q = r.standard_normal((B, Hq, L, D))
+    k = r.standard_normal((B, Hkv, L, D))
+    v = r.standard_normal((B, Hkv, L, D))
+    budgets = [4, 6]
+    s = 1.0 / math.sqrt(D)
+    want_sc = np.zeros((B, Hkv, L))
+    for h in range(Hq):
+        g = h // G
+        for p in range(L - W, L):
+            logits = [s * sum(q[0, h, p, d] * k[0, g, j, d] for d in range(D)) for j in range(p + 1)]
+            mx = max(logits)
+            e = [math.exp(x - mx) for x in logits]
+            z = sum(e)
+            for j in range(p + 1):
+                want_sc[0, g, j] += e[j] / z
+    sc, perm, out = O.forward(q, k, v, W, budgets)
+    np.testing.assert_allclose(sc, want_sc, rtol=1e-13, atol=1e-15)
+    s32 = want_sc.astype(np.float32)
+    for g, K in enumerate(budgets):
+        kept = _brute_force_topk([float(x) for x in s32[0, g]], K)
+        assert perm[0, g, :K].tolist() == kept
+        assert perm[0, g, K:].tolist() == sorted(set(range(L)) - set(kept))
+        keep = np.zeros(L, bool)
+        keep[kept] = True
+        mask = keep[None, :] & (np.arange(L)[None, :] <= np.arange(L)[:, None])
+        hs = slice(g * G, (g + 1) * G)
+        ref = _sdpa64(q[:, hs], k[:, g:g + 1], v[:, g:g + 1], mask=mask)
+        np.testing.assert_allclose(out[0, hs][:, keep], ref[0][:, keep], rtol=0, atol=1e-12)
+        assert np.all(out[0, hs][:, ~keep] == 0.0)
