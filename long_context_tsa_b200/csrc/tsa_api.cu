@@ -27,11 +27,12 @@ int window_rows_padded(const Dims& d, int window) {
   return (M + 63) / 64 * 64;
 }
 
+// Key-range splits per KV head of the SIMT score passes.  A function of L only:
+// a KV head's scores do not depend on which other heads share the call, so a
+// layer split by KV group across calls (or GPUs) gives bit-identical scores.
 int score_splits(const Dims& d) {
   const int ntiles = (d.L + kScoreKeyTile - 1) / kScoreKeyTile;
-  const int groups = d.B * d.Hkv;
-  const int want = (2 * 148 + groups - 1) / groups;
-  int s = want < ntiles ? want : ntiles;
+  int s = ntiles < 74 ? ntiles : 74;
   s = s < kMaxScoreSplits ? s : kMaxScoreSplits;
   return s < 1 ? 1 : s;
 }

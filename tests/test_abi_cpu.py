@@ -154,11 +154,17 @@ def test_zero_dropped_and_noalloc_reject_before_launch(lib):
         N.STATUS["TSA_ERR_UNSUPPORTED"]
     # The no-allocation scorer checks the shape, then its fixed scratch, then the pointers:
     # B = 65 with 32/8 heads and window 64 needs more than its 1 MiB, whatever the pointers.
-    for dt in (N.TSA_BF16, N.TSA_F32):
-        big = N.make_desc(B=65, Hq=32, Hkv=8, L=8192, D=128, dtype=dt)
+    # At the shortest lengths (one split: L <= 128 in bf16, L <= 64 in f32) B = 64 fills it exactly.
+    for dt, L_fit in ((N.TSA_BF16, 128), (N.TSA_F32, 64)):
+        big = N.make_desc(B=65, Hq=32, Hkv=8, L=L_fit, D=128, dtype=dt)
         assert lib.tsa_score_noalloc(ctypes.byref(big), None, None, 64, None, None) == wsz
-        fits = N.make_desc(B=64, Hq=32, Hkv=8, L=256, D=128, dtype=dt)
+        fits = N.make_desc(B=64, Hq=32, Hkv=8, L=L_fit, D=128, dtype=dt)
         assert lib.tsa_score_noalloc(ctypes.byref(fits), None, None, 64, None, None) == inv
+        two_splits = N.make_desc(B=64, Hq=32, Hkv=8, L=2 * L_fit, D=128, dtype=dt)
+        assert lib.tsa_score_noalloc(ctypes.byref(two_splits), None, None, 64, None, None) == wsz
+    # The bf16 128K layer (8 KV heads x 37 splits x 256 rows x 8 bytes = 606 KB) fits.
+    layer = N.make_desc(B=1, Hq=32, Hkv=8, L=131072, D=128, dtype=N.TSA_BF16)
+    assert lib.tsa_score_noalloc(ctypes.byref(layer), None, None, 64, None, None) == inv
     assert lib.tsa_score_noalloc(ctypes.byref(desc(D=96)), None, None, 64, None, None) == \
         N.STATUS["TSA_ERR_UNSUPPORTED"]
     assert lib.tsa_score_noalloc(ctypes.byref(desc()), None, None, 65, None, None) == \

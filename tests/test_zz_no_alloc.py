@@ -70,20 +70,27 @@ def test_noalloc_score_matches_oracle_and_tsa_score_on_two_calls_in_a_row():
 
 
 def test_noalloc_score_fills_the_whole_array_at_its_limit():
-    # 32/8 heads, window 64, B = 64: the partials take exactly the 1 MiB array
-    # (512 KV heads x 1 split x 256 window rows x 8 bytes) in both dtypes.
-    for dtype, D in (("bf16", 128), ("f32", 64)):
-        w = I.custom("noalloc_limit", B=64, Hq=32, Hkv=8, L=256, D=D, dtype=dtype, W=64, sigma=0.5)
+    # 32/8 heads, window 64, B = 64 at the shortest length with one key split (L = 128
+    # in bf16, L = 64 in f32): the partials take exactly the 1 MiB array
+    # (512 KV heads x 1 split x 256 window rows x 8 bytes).
+    for dtype, D, L in (("bf16", 128, 128), ("f32", 64, 64)):
+        w = I.custom("noalloc_limit", B=64, Hq=32, Hkv=8, L=L, D=D, dtype=dtype, W=64, sigma=0.5)
         _check(w, seed=3, with_oracle=False)
+
+
+def test_noalloc_score_bench_layer():
+    # The 128K bf16 layer (8 KV heads x 37 splits x 256 rows x 8 bytes = 606 KB) fits.
+    w = I.WORKLOADS["gqa_bf16_L131072"]
+    _check(w, seed=4, with_oracle=False)
 
 
 def test_noalloc_score_refuses_shapes_beyond_its_fixed_scratch():
     # B = 65 needs more than the 1 MiB array: refused with TSA_ERR_WORKSPACE before
     # the (null) pointers are looked at, so nothing can be launched.
-    for dtype in (N.TSA_BF16, N.TSA_F32):
-        big = N.make_desc(B=65, Hq=32, Hkv=8, L=8192, D=128, dtype=dtype)
+    for dtype, L in ((N.TSA_BF16, 128), (N.TSA_F32, 64)):
+        big = N.make_desc(B=65, Hq=32, Hkv=8, L=L, D=128, dtype=dtype)
         assert N.lib().tsa_score_noalloc(ctypes.byref(big), None, None, 64, None, None) == \
             N.STATUS["TSA_ERR_WORKSPACE"]
-        fits = N.make_desc(B=64, Hq=32, Hkv=8, L=256, D=128, dtype=dtype)
+        fits = N.make_desc(B=64, Hq=32, Hkv=8, L=L, D=128, dtype=dtype)
         assert N.lib().tsa_score_noalloc(ctypes.byref(fits), None, None, 64, None, None) == \
             N.STATUS["TSA_ERR_INVALID_ARG"]
