@@ -444,9 +444,16 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {T.tsa_status_string(st)}")
 
-    # L2 (126 MB) is flushed between timed steps by writing a 256 MB buffer; each step
-    # is timed by its own events, so the flushes sit outside the step times.
+    # L2 (126 MB) is flushed between timed steps: a 256 MB buffer is written, then
+    # another 256 MB buffer is read, so the step starts on a cold L2 that holds no
+    # dirty lines to write back.  Each step is timed by its own events, so the
+    # flushes sit outside the step times.
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -459,7 +466,7 @@ def main():
     launches0 = T.tsa_debug_launch_count()
     start.record(stream)
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -527,7 +534,7 @@ def main():
                    "block_density": args.density if block_sparse else None,
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D, "W": w.W,
                    "K_per_kv_head": budgets,
-                   "l2": ("flushed between timed steps (a 256 MB buffer written outside the per-step events); "
+                   "l2": ("flushed between timed steps (256 MB written, then 256 MB read, outside the per-step events); "
                           f"inputs also exceed L2: q {q.numel() * q.element_size() / 1e9:.2f} GB, "
                           f"k and v {k.numel() * k.element_size() / 1e6:.0f} MB each"),
                    "timed_loop_ms_incl_flushes": loop_ms,
