@@ -34,6 +34,17 @@ What it computes (each function cites the passage it follows):
   128 x 128 blocks of the compressed (query, key) space.  Source: the
   sciencestack page, Figures 1 and 5b (Token Sparse Attention composed with a
   block-sparse attention kernel inside the compressed token set).
+* ``out_proj_residual`` -- the output projection of the attention output,
+  added to the residual.  Source: the skill page, Step 3
+  (``SparseAttentionHead.forward``: ``out_proj`` on the attention output of
+  the selected tokens, then ``scatter_attention_output`` back to full length);
+  the sciencestack page, Figure 3 (outputs scattered back into the full
+  sequence layout before the residual connection is added).  Reading: the
+  projection is a bias-free linear map of the heads' outputs concatenated per
+  position (the multi-head form of the page's single-head ``out_proj``); a row
+  dropped by a head's group contributes zero, so projecting the compressed rows
+  and scattering them equals projecting the scattered rows; the residual is
+  added to every row, as in Figure 3.
 * ``drift``   -- representation drift between two hidden-state tensors:
   one minus the mean, over all (batch, position) rows, of the cosine of the
   two rows after each is divided by max(its L2 norm, eps).  Source: the skill
@@ -79,6 +90,7 @@ __all__ = [
     "attend_accumulate",
     "attend_block_sparse",
     "BLOCK",
+    "out_proj_residual",
     "forward",
     "row_cosine",
     "drift",
@@ -342,6 +354,25 @@ def attend_accumulate(base, q, k, v, perm, budgets, scale=None) -> np.ndarray:
             K = int(kept[b * Hkv + g])
             out[b, h, perm[b, g, :K]] += attend_rows(q, k, v, perm[b, g], K, b, h, G, np.arange(K), scale)
     return out
+
+
+def out_proj_residual(x, attn_out, w_o, b: int = 0, rows=None) -> np.ndarray:
+    """Residual plus the output projection of the full-length attention output.
+
+    x [B, L, N] is the residual stream, attn_out [B, Hq, L, D] the attention
+    output as ``attend`` writes it (zeros at every row a head's KV group
+    dropped), w_o [N, Hq * D] the projection weight in the layout of an
+    ``nn.Linear`` weight (out_features x in_features), no bias.  For batch
+    entry ``b`` and positions ``rows`` (default: all) returns, as float64
+    [len(rows), N],
+        x[b, p, :] + concat_h(attn_out[b, h, p, :]) @ w_o.T
+    -- the skill page's Step 3 ``out_proj`` followed by the scatter back to
+    full length, and Figure 3's residual add after the scatter.
+    """
+    B, Hq, L, D = np.shape(attn_out)
+    rows = np.arange(L) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.transpose(_f64(np.asarray(attn_out)[b][:, rows, :]), (1, 0, 2)).reshape(rows.size, Hq * D)
+    return _f64(np.asarray(x)[b][rows]) + o @ _f64(w_o).T
 
 
 def forward(q, k, v, window: int, budgets, scale=None):

@@ -630,3 +630,66 @@ def test_forward_matches_independent_construction():
         ref = _sdpa64(q[:, hs], k[:, g:g + 1], v[:, g:g + 1], mask=mask)
         np.testing.assert_allclose(out[0, hs][:, keep], ref[0][:, keep], rtol=0, atol=1e-12)
         assert np.all(out[0, hs][:, ~keep] == 0.0)
+
+
+# --- output projection + residual (skill page Step 3, sciencestack Figure 3) ----------------
+
+
+def _compress_project_scatter(x, attn_out, w_o, perm, budgets):
+    # The page's order written out per head: gather the kept rows (the compressed
+    # output), project them with the head's slice of the weight, scatter-add back.
+    B, Hq, L, D = attn_out.shape
+    Hkv = perm.shape[1]
+    G = Hq // Hkv
+    y = np.array(x, dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            K = min(budgets[b * Hkv + g], L)
+            idx = perm[b, g, :K]
+            comp = attn_out[b, h, idx, :]  # [K, D]
+            proj = np.zeros((K, w_o.shape[0]))
+            for i in range(K):
+                for n in range(w_o.shape[0]):
+                    proj[i, n] = sum(comp[i, d] * w_o[n, h * D + d] for d in range(D))
+            y[b, idx, :] += proj
+    return y
+
+
+def test_out_proj_is_compress_project_scatter_and_torch_linear():
+    r = np.random.default_rng(91)
+    B, Hq, Hkv, L, D, N = 1, 4, 2, 12, 4, 6
+    budgets = [5, 8]
+    perm = O.select(r.random((B, Hkv, L)), budgets)
+    attn = r.standard_normal((B, Hq, L, D))
+    for g in range(Hkv):  # zeros at the rows each group dropped, as attend writes them
+        attn[0, g * 2:(g + 1) * 2, perm[0, g, budgets[g]:], :] = 0.0
+    x = r.standard_normal((B, L, N))
+    w = r.standard_normal((N, Hq * D))
+    got = O.out_proj_residual(x, attn, w)
+    np.testing.assert_allclose(got, _compress_project_scatter(x, attn, w, perm, budgets)[0], rtol=0, atol=1e-12)
+    o = torch.from_numpy(attn[0]).permute(1, 0, 2).reshape(L, Hq * D)
+    ref = torch.from_numpy(x[0]) + torch.nn.functional.linear(o, torch.from_numpy(w))
+    np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
+    # A row no group keeps is the residual, bit for bit; a row subset equals those rows.
+    kept_any = np.zeros(L, bool)
+    for g in range(Hkv):
+        kept_any[perm[0, g, :budgets[g]]] = True
+    np.testing.assert_array_equal(got[~kept_any], x[0][~kept_any])
+    rows = np.array([0, 3, 11])
+    np.testing.assert_array_equal(O.out_proj_residual(x, attn, w, rows=rows), got[rows])
+
+
+def test_out_proj_identity_weight_and_zero_attention():
+    r = np.random.default_rng(92)
+    B, Hq, L, D = 2, 2, 5, 3
+    attn = r.standard_normal((B, Hq, L, D))
+    x = r.standard_normal((B, L, Hq * D))
+    eye = np.eye(Hq * D)
+    for b in range(B):
+        # Identity weight: the heads' outputs concatenated per position, added to x.
+        want = x[b] + np.concatenate([attn[b, h] for h in range(Hq)], axis=1)
+        np.testing.assert_array_equal(O.out_proj_residual(x, attn, eye, b=b), want)
+        # No attention output: the residual comes back unchanged.
+        w = r.standard_normal((Hq * D, Hq * D))
+        np.testing.assert_array_equal(O.out_proj_residual(x, np.zeros_like(attn), w, b=b), x[b])
