@@ -148,6 +148,33 @@ def time_zero_dropped(T, w, desc, perm, budgets, out, ws, stream, dev, peaks, pe
             "note": f"{dropped} dropped rows x {w.G} query heads; timed alone, {reps} launches back to back"}
 
 
+def out_proj_roofline(w, budgets, perm, t_ms, peaks, peak_src):
+    """tsa_out_proj against the tensor-core peak on its useful flops: every kept
+    (position, KV group) row times the group's G*D columns of W_o times hidden,
+    2 flops per multiply-add; beside it the HBM bytes of the rows it must touch
+    (the residual rows of positions any group kept, read and written, and the
+    kept attention rows read once)."""
+    hidden = w.Hq * w.D
+    kept = [min(int(x), w.L) for x in budgets]
+    flops = 2.0 * sum(kept) * w.G * w.D * hidden
+    pm = perm.cpu().numpy()
+    union = 0
+    for b in range(w.B):
+        m = np.zeros(w.L, bool)
+        for g in range(w.Hkv):
+            m[pm[b, g, :kept[b * w.Hkv + g]]] = True
+        union += int(m.sum())
+    esz = 2 if w.dtype == "bf16" else 4
+    nbytes = union * hidden * esz * 2 + sum(kept) * w.G * w.D * esz
+    a = flops / (t_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    return {"kernel": "out_proj (mask sort + op_tc: projection of the kept rows + residual)", "bound": "tensor",
+            "achieved": a, "peak": peak, "unit": "TFLOP/s", "frac": a / peak, "ms": t_ms, "useful_flops": flops,
+            "hbm_bytes": nbytes, "hbm_frac": nbytes / (t_ms * 1e-3) / 1e9 / hbm, "positions_kept_by_any_group": union,
+            "peak_source": f"bf16_tflops ({peak_src}); hbm_gbs for hbm_frac"}
+
+
 def capture_note(src):
     """Provenance of a traffic figure read from a committed ncu summary."""
     if not src:
@@ -354,13 +381,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op", default="forward",
-                    choices=["forward", "forward-accumulate", "forward-coverage", "forward-block-sparse", "drift",
-                             "sweep"],
+                    choices=["forward", "forward-accumulate", "forward-coverage", "forward-block-sparse",
+                             "forward-out-proj", "drift", "sweep"],
                     help="forward: score/select/attend (the headline); forward-accumulate: the same with the "
                          "scatter-add attention into a resident output; forward-coverage: budgets chosen per KV "
                          "head from the coverage --tau (one device-to-host copy of the budgets per step); "
                          "forward-block-sparse: attention restricted by a 128 x 128 block mask of --density in the "
-                         "compressed space; drift: the representation-drift pass; sweep: the sparsity sweep at "
+                         "compressed space; forward-out-proj: the forward followed by the output projection of the "
+                         "attention output added to a resident residual (tsa_out_proj, hidden = Hq * D); drift: the "
+                         "representation-drift pass; sweep: the sparsity sweep at "
                          "128K against dense causal attention in the same library (K = L)")
     ap.add_argument("--density", type=float, default=0.5, help="block density for --op forward-block-sparse")
     ap.add_argument("--tau", type=float, default=0.005, help="token coverage for --op forward-coverage")
@@ -408,6 +437,13 @@ def main():
     accumulate = args.op == "forward-accumulate"
     coverage = args.op == "forward-coverage"
     block_sparse = args.op == "forward-block-sparse"
+    out_proj = args.op == "forward-out-proj"
+    if out_proj:  # the residual stream and a seeded projection weight (hidden = Hq * D)
+        hidden = w.Hq * w.D
+        gx = torch.Generator(device=dev).manual_seed(1000 + rank)
+        x_res = torch.randn((w.B, w.L, hidden), generator=gx, device=dev).to(q.dtype)
+        w_o = (torch.randn((hidden, hidden), generator=gx, device=dev) / math.sqrt(hidden)).to(q.dtype)
+        op_ws = T.alloc_out_proj_workspace(desc, device=dev)
     bm_host = block_mask_for(w, args.density) if block_sparse else None
     bm_dev = torch.from_numpy(bm_host).to(dev) if block_sparse else None
     if accumulate:
@@ -436,6 +472,10 @@ def main():
             T.tsa_attend(desc, q, k, v, perm, budgets, out, ws)
         if ev is not None:
             ev[3].record(stream)
+        if out_proj:
+            T.tsa_out_proj(desc, out, perm, budgets, w_o, x_res, op_ws)
+            if ev is not None:
+                ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -454,7 +494,8 @@ def main():
     def flush_l2():
         flush.zero_()
         flush_rd.sum()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    last = 4 if out_proj else 3  # the event that ends a step
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -479,7 +520,7 @@ def main():
         raise RuntimeError(f"device status after timing: {T.tsa_status_string(st)}")
 
     loop_ms = start.elapsed_time(end)  # includes the flushes
-    steps_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    steps_ms = sum(e[0].elapsed_time(e[last]) for e in evs)
     t_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     t_attend = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -494,6 +535,12 @@ def main():
     peak = float(peaks["bf16_tflops"])
     traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
                                                                        "long_context_tsa_b200/csrc/tc_ptx.cuh"])
+    op_line = None
+    if out_proj:
+        if T.tsa_check_status(op_ws) != 0:
+            raise RuntimeError("device status of the output projection")
+        t_op = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+        op_line = out_proj_roofline(w, budgets, perm, t_op, peaks, peak_src)
     zf = None
     if not coverage:
         zf = time_zero_dropped(T, w, desc, perm, budgets, out, ws, stream, dev, peaks, peak_src, args.workload)
@@ -540,13 +587,15 @@ def main():
                    "timed_loop_ms_incl_flushes": loop_ms,
                    "parallelism": f"{world} independent layers, one per GPU",
                    "input_checksum": input_checksum(q, k, v)},
-        "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend},
+        "breakdown_ms": {"score": t_score, "select": t_select, "attend": t_attend,
+                         **({"out_proj": op_line["ms"]} if op_line else {})},
         "attend_tflops": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"bf16_tflops ({peak_src})",
                      "kernel": "attend_tc (tsa_attend: gather + attention + scatter + zero fill)",
                      "traffic_source": traffic_src, "traffic_capture": capture_note(traffic_src)},
-        "rooflines_other": other_rooflines(w, t_score, t_select, peaks, peak_src) + ([zf] if zf else []),
+        "rooflines_other": other_rooflines(w, t_score, t_select, peaks, peak_src) + ([zf] if zf else []) +
+        ([op_line] if op_line else []),
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,

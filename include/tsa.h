@@ -128,6 +128,38 @@ TSA_API tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k
                       size_t ws_bytes, void* stream);
 
 /*
+ * tsa_out_proj -- the attention output's projection added to the residual
+ * ("Token Sparse Attention Long Context" skill page, Step 3: out_proj applied
+ * to the attention output of the selected tokens, then scattered back to full
+ * length; [P2] Figure 3: the residual connection is added after the scatter):
+ *   x[b, p, :] += sum over query heads h whose KV group g = h / G kept p of
+ *                 attn_out[b, h, p, :] . w_o[:, h*D : (h+1)*D]^T
+ * for every position p kept by at least one group; rows no group kept are
+ * left untouched.  The projection is bias-free (the multi-head form of the
+ * page's out_proj on the concatenated head outputs).
+ *   attn_out: device [B, Hq, L, D] in desc->dtype, the layout tsa_attend
+ *             writes; rows at positions a head's group dropped are not read.
+ *   perm, budget_host: the selection tsa_select produced (same rules as
+ *             tsa_attend).
+ *   w_o:      device [hidden, Hq*D] row-major in desc->dtype (an nn.Linear
+ *             weight, out_features x in_features).
+ *   x:        device [B, L, hidden] in desc->dtype, holding the residual on
+ *             entry; read and written in place (fp32 accumulation, one
+ *             rounding to the dtype per element).
+ *   ws:       device workspace of tsa_out_proj_workspace_size() bytes, 16-byte
+ *             aligned, status word first (tsa_check_status reads it).
+ * Supported: Hkv <= 16 per batch entry; hidden a multiple of 256 for bf16
+ * (tcgen05 kernel), of 64 for f32 (SIMT kernel).  One memset and five kernel
+ * launches on `stream`; returns after enqueueing.  TSA_ERR_INVALID_ARG for a
+ * bad pointer, budget or hidden; TSA_ERR_UNSUPPORTED outside the shapes;
+ * TSA_ERR_WORKSPACE for a short workspace.
+ */
+TSA_API size_t tsa_out_proj_workspace_size(const tsa_desc* desc);
+TSA_API tsa_status tsa_out_proj(const tsa_desc* desc, const void* attn_out, const int32_t* perm,
+                                const int32_t* budget_host, const void* w_o, int32_t hidden, void* x, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
  * tsa_zero_dropped -- the zero rows of the scatter on their own ([P1] Step 2
  * scatter_attention_output builds the full-length output from zeros; [P2]
  * Figure 3 scatters into the full sequence layout): for each (b, g) with

@@ -12,6 +12,7 @@ from ._native import (  # noqa: F401
     TsaDesc,
     TsaError,
     alloc_drift_workspace,
+    alloc_out_proj_workspace,
     alloc_workspace,
     desc_for,
     make_desc,
@@ -29,6 +30,8 @@ from ._native import (  # noqa: F401
     tsa_forward_coverage,
     tsa_forward_host,
     tsa_layer_stable,
+    tsa_out_proj,
+    tsa_out_proj_workspace_size,
     tsa_score,
     tsa_score_noalloc,
     tsa_select,

@@ -24,7 +24,8 @@ EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
-            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2", "tsa_zero_dropped")
+            "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2", "tsa_zero_dropped",
+            "tsa_out_proj_workspace_size", "tsa_out_proj")
 
 
 class TsaDesc(ctypes.Structure):
@@ -59,6 +60,8 @@ _SIGS = {
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
+    "tsa_out_proj_workspace_size": (_SZ, [ctypes.POINTER(TsaDesc)]),
+    "tsa_out_proj": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
     "tsa_zero_dropped": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _SZ, _P]),
     "tsa_debug_exp2": (ctypes.c_int, [_P, _P, _I32, _P]),
     "tsa_attend_block_sparse": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -149,6 +152,26 @@ def tsa_select(desc, scores, budgets, perm, ws, stream=None):
 def tsa_attend(desc, q, k, v, perm, budgets, out, ws, stream=None):
     _check(lib().tsa_attend(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(perm), _budgets(budgets),
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "tsa_attend")
+
+
+def tsa_out_proj_workspace_size(desc) -> int:
+    return int(lib().tsa_out_proj_workspace_size(ctypes.byref(desc)))
+
+
+def alloc_out_proj_workspace(desc, device="cuda") -> torch.Tensor:
+    n = tsa_out_proj_workspace_size(desc)
+    if n == 0:
+        raise TsaError(STATUS["TSA_ERR_UNSUPPORTED"], "tsa_out_proj_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def tsa_out_proj(desc, attn_out, perm, budgets, w_o, x, ws, stream=None):
+    """x[b, p, :] += the projection (w_o, [hidden, Hq*D]) of the heads' attention rows kept at p."""
+    hidden = int(w_o.shape[0])
+    if x.shape[-1] != hidden or w_o.shape[1] != desc.Hq * desc.D:
+        raise ValueError("x must be [B, L, hidden] and w_o [hidden, Hq*D]")
+    _check(lib().tsa_out_proj(ctypes.byref(desc), _ptr(attn_out), _ptr(perm), _budgets(budgets), _ptr(w_o), hidden,
+                              _ptr(x), _ptr(ws), ws.numel(), _stream(stream)), "tsa_out_proj")
 
 
 def tsa_zero_dropped(desc, perm, budgets, out, ws, stream=None):

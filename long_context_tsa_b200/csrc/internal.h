@@ -71,6 +71,16 @@ cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const 
                              const uint8_t* block_mask, cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
+// Output projection (out_proj.cu): its own workspace, a 256-byte status header
+// first, then the group masks of the positions and their counting sort.
+constexpr int kOutProjMaxHkv = 16;  // the sort has one bucket per mask: 2^Hkv
+struct OpWsLayout {
+  size_t count, mask, hist, zero_end;  // [count, zero_end) is zeroed by each call
+  size_t cursor, order, key, total;
+};
+OpWsLayout out_proj_ws_layout(const Dims& d);
+cudaError_t launch_out_proj(const Dims& d, const void* attn, const int32_t* perm, const Budgets& kept,
+                            const void* w_o, int N, void* x, void* ws, cudaStream_t st);
 constexpr int kDriftMaxBlocks = 2048;  // drift partials held in its workspace
 constexpr size_t kDriftWsBytes = 256 + sizeof(double) * kDriftMaxBlocks;
 int drift_grid(int64_t rows);

@@ -228,6 +228,29 @@ tsa_status tsa_attend(const tsa_desc* desc, const void* q, const void* k, const 
   return run_attend(d, q, k, v, perm, kb, out, ws, static_cast<cudaStream_t>(stream));
 }
 
+size_t tsa_out_proj_workspace_size(const tsa_desc* desc) {
+  Dims d;
+  if (check_desc(desc, &d) != TSA_OK || d.Hkv > kOutProjMaxHkv) return 0;
+  return out_proj_ws_layout(d).total;
+}
+
+tsa_status tsa_out_proj(const tsa_desc* desc, const void* attn_out, const int32_t* perm, const int32_t* budget_host,
+                        const void* w_o, int32_t hidden, void* x, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  tsa_status s = check_desc(desc, &d);
+  if (s != TSA_OK) return s;
+  if (d.Hkv > kOutProjMaxHkv) return TSA_ERR_UNSUPPORTED;
+  if (hidden < 1) return TSA_ERR_INVALID_ARG;
+  if (hidden % (d.dtype == TSA_BF16 ? 256 : 64) != 0) return TSA_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.L * hidden >= (1LL << 40)) return TSA_ERR_UNSUPPORTED;
+  if (!aligned16(attn_out) || !aligned16(perm) || !aligned16(w_o) || !aligned16(x) || !aligned16(ws))
+    return TSA_ERR_INVALID_ARG;
+  if (ws_bytes < out_proj_ws_layout(d).total) return TSA_ERR_WORKSPACE;
+  Budgets kb;
+  if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
+  return cuda_status(launch_out_proj(d, attn_out, perm, kb, w_o, hidden, x, ws, static_cast<cudaStream_t>(stream)));
+}
+
 tsa_status tsa_zero_dropped(const tsa_desc* desc, const int32_t* perm, const int32_t* budget_host, void* out,
                             void* ws, size_t ws_bytes, void* stream) {
   Dims d;
