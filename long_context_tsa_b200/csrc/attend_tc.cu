@@ -91,7 +91,6 @@ struct Cfg {
   static constexpr int SMEM = OFF_ZERO + D * 2 + 1024;  // + alignment slack
   static constexpr int CPR = D / 8;    // 16-byte chunks per row
   static constexpr int RPI = 32 / CPR;  // rows per warp-wide copy instruction
-  static constexpr int DEFER = 2;       // copy groups left in flight before a group is published
   static constexpr uint32_t O_COL0 = 256u;  // S_t lives at column 128 * t
 };
 
@@ -163,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 32 * kProducerWarps);  // every producer lane publishes its own copies
+    mbar_init(bar_q, 32 * kProducerWarps);  // every producer lane arrives once its own copies land
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar_full(s), 32 * kProducerWarps);
       mbar_init(bar_empty(s), 1);
@@ -196,11 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     // ------------------------------------------------------------ producer
     // Copies are 16-byte cp.async chunks written straight into the 128-byte
     // swizzled K-major layout the MMA reads; one warp instruction moves RPI
-    // whole rows.  Each tile is one commit group; a group is published (proxy
-    // fence, then an arrive by every lane) once DEFER newer groups are in
-    // flight.  Groups 0 and 1 hold the Q tiles (-> bar_q); group 2 + i holds
-    // load i of the ring (K_0, V_0, K_1, ...; fill i / NS of stage i % NS).
-    // With DEFER < NS the load a slot waits for is always published first.
+    // whole rows.  After issuing a tile every lane arrives on the tile's
+    // barrier through cp.async.mbarrier.arrive, which fires once the lane's
+    // copies have landed: no lane waits for its own copies, so loads of every
+    // free ring stage are in flight at once.  The Q tiles arrive on bar_q, ring
+    // load i (K_0, V_0, K_1, ...) on full[i % NS]; the MMA thread makes the
+    // landed rows visible to the tensor core (proxy fence) after its wait.
     const int pw = warp - kProducerWarp0;  // this warp owns rows [32 pw, 32 pw + 32) of every tile
     const int my_c = lane % C::CPR, my_r = lane / C::CPR;
     const uint32_t chunk_off = (uint32_t)(my_c >> 3) * 16384u;
@@ -211,15 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         const __nv_bfloat16* g = src + (size_t)tab[row] * D + my_c * 8;
         cp_async16(dst + chunk_off + row * 128 + ((((uint32_t)my_c & 7u) ^ ((uint32_t)row & 7u)) << 4), g);
       }
-      cp_async_commit();
-    };
-    auto publish_q = [&]() {  // both Q tiles have landed in shared memory
-      fence_proxy_async_smem();
-      mbar_arrive(bar_q);
-    };
-    auto publish_ring = [&](int r) {  // ring load r has landed
-      fence_proxy_async_smem();
-      mbar_arrive(bar_full(r % C::NS));
     };
     // Row tables: lane l owns row 32 pw + l of each tile (the warp reads only its rows).
     const int my_row = 32 * pw + lane;
@@ -230,14 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       qtab[t * 128 + my_row] = (b * p.Hq + g * p.G + hh) * L + load_pos(pm, pos, L, p.status);
     }
     __syncwarp();
-    issue_tile(sQ, p.q, qtab);                      // group 0
-    issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);   // group 1
-    int committed = 2;  // groups 0, 1: Q tiles; group 2 + r: ring load r
+    issue_tile(sQ, p.q, qtab);
+    issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);
+    cp_async_mbar_arrive(bar_q);
     const int kv_row0 = (b * p.Hkv + g) * L;
     int kt_load = next_active(-1);  // the active tile whose rows y_next holds
     int y_next = kv_row0 + load_pos(pm, min(min(kt_load, n_kt - 1) * 128 + my_row, K - 1), L, p.status);
-    int published = 0;  // ring loads published so far
-    bool q_published = false;
     for (int i = 0; i < 2 * n_act; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int s = i % C::NS;
@@ -256,18 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         }
       }
       issue_tile(sKV + s * C::KV_BYTES, (i & 1) ? p.v : p.k, kvtab);
-      ++committed;
-      // Publish what has landed, keeping DEFER groups in flight.
-      cp_async_wait<C::DEFER>();  // groups [0, committed - DEFER) have landed
-      if (!q_published && committed - C::DEFER >= 2) {
-        publish_q();
-        q_published = true;
-      }
-      while (2 + published < committed - C::DEFER) publish_ring(published++);
+      cp_async_mbar_arrive(bar_full(s));
     }
-    cp_async_wait_all();
-    if (!q_published) publish_q();
-    while (2 + published < committed) publish_ring(published++);
+    cp_async_wait_all();  // no copy is still writing shared memory when the CTA exits
   } else if (warp >= kZeroWarp0) {
     // ------------------------------------------------------------ zero fill
     const int U = p.zero_fill ? L - K : 0;  // dropped rows of this group left to this kernel
@@ -300,8 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16(128, D, 0, 1);
       bool ok = mbar_wait(bar_q, 0, p.wait_limit, abort_flag);
+      fence_proxy_async_smem();  // rows landed by cp.async (generic proxy) are read by the tensor core
       auto wait_load = [&](int i) -> bool {
-        return mbar_wait(bar_full(i % C::NS), (i / C::NS) & 1, p.wait_limit, abort_flag);
+        const bool got = mbar_wait(bar_full(i % C::NS), (i / C::NS) & 1, p.wait_limit, abort_flag);
+        fence_proxy_async_smem();
+        return got;
       };
       auto qk = [&](int t, int i_k) {
         const uint32_t kbase = sKV + (i_k % C::NS) * C::KV_BYTES;

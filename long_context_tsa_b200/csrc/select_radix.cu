@@ -40,8 +40,13 @@ constexpr int kClusterCtas = 8;
 constexpr int kThreads = 1024;
 constexpr int kPerThread = 4;
 constexpr int kChunk = kThreads * kPerThread;
+// A CTA's slice of sortable keys is staged in shared memory once when it holds
+// at most this many (160 KB): every radix pass, the counts and the compaction
+// then read shared memory instead of the scores in L2.
+constexpr int kMaxStagedKeys = 40960;
 
 struct SelectArgs {
+  int staged;         // 1: the slice's keys are in dynamic shared memory
   const float* scores;
   int32_t* perm;
   uint32_t* status;
@@ -63,6 +68,10 @@ __device__ __forceinline__ uint64_t token_mass(float s, float mass_scale) {
   if ((bits >> 23) == 0u || k <= -24) return 0u;  // zero, subnormal or below 1: floor is 0
   const uint64_t sig = (bits & 0x7FFFFFu) | 0x800000u;
   return k >= 0 ? sig << k : sig >> -k;
+}
+
+__device__ __forceinline__ void hist_add(uint32_t* h, bool match, uint32_t dg) {
+  if (match) atomicAdd(&h[dg], 1u);
 }
 
 __device__ __forceinline__ float key_to_float(uint32_t key) {
@@ -127,7 +136,7 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return before;
 }
 
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads, 1)
     select_radix(SelectArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -142,6 +151,12 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   const int hi = min(L, lo + per);
   const int tid = threadIdx.x;
 
+  extern __shared__ uint32_t skeys[];  // [hi - lo] order keys when a.staged
+  if (a.staged) {
+    for (int i = lo + tid; i < hi; i += kThreads) skeys[i - lo] = order_key(sc[i]);
+    __syncthreads();
+  }
+  auto key_at = [&](int i) -> uint32_t { return a.staged ? skeys[i - lo] : order_key(sc[i]); };
   __shared__ uint32_t hist[2][256];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t dig_warp[8];
@@ -159,7 +174,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
     if (tid == 0) sh_mass = 0u;
     __syncthreads();
     uint64_t my = 0u;
-    for (int i = lo + tid; i < hi; i += kThreads) my += token_mass(sc[i], a.mass_scale);
+    for (int i = lo + tid; i < hi; i += kThreads) my += token_mass(key_to_float(key_at(i)), a.mass_scale);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) my += __shfl_xor_sync(0xffffffffu, my, o);
     if ((tid & 31) == 0 && my) atomicAdd(reinterpret_cast<unsigned long long*>(&sh_mass), (unsigned long long)my);
@@ -184,12 +199,12 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
         }
         __syncthreads();
         for (int i = lo + tid; i < hi; i += kThreads) {
-          const float f = sc[i];
-          const uint32_t key = order_key(f);
-          if ((key & mask) == prefix) {
-            const uint32_t dg = (key >> shift) & 255u;
-            atomicAdd(&hc[dg], 1u);
-            const uint64_t m = token_mass(f, a.mass_scale);
+          const uint32_t key = key_at(i);
+          const bool match = (key & mask) == prefix;
+          const uint32_t dg = (key >> shift) & 255u;
+          hist_add(hc, match, dg);
+          if (match) {
+            const uint64_t m = token_mass(key_to_float(key), a.mass_scale);
             const uint32_t mlo = (uint32_t)m;
             uint32_t mhi = (uint32_t)(m >> 32);
             if (mlo) {
@@ -250,8 +265,8 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
       if (tid < 256) h[tid] = 0u;
       __syncthreads();
       for (int i = lo + tid; i < hi; i += kThreads) {
-        const uint32_t key = order_key(sc[i]);
-        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        const uint32_t key = key_at(i);
+        hist_add(h, (key & mask) == prefix, (key >> shift) & 255u);
       }
       cluster.sync();
       if (tid < 256) {
@@ -290,7 +305,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   if (partial) {
     uint32_t gt = 0u, eq = 0u;
     for (int i = lo + tid; i < hi; i += kThreads) {
-      const uint32_t key = order_key(sc[i]);
+      const uint32_t key = key_at(i);
       gt += key > T;
       eq += key == T;
     }
@@ -320,7 +335,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
       iseq[e] = 0u;
       if (i < hi) {
         if (partial) {
-          const uint32_t key = order_key(sc[i]);
+          const uint32_t key = key_at(i);
           isgt[e] = key > T;
           iseq[e] = key == T;
         } else {
@@ -356,6 +371,19 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
+cudaError_t launch_radix(const Dims& d, SelectArgs& a, cudaStream_t st) {
+  const int per = (d.L + kClusterCtas - 1) / kClusterCtas;
+  a.staged = per <= kMaxStagedKeys ? 1 : 0;
+  const int smem = a.staged ? per * (int)sizeof(uint32_t) : 0;
+  cudaError_t e = cudaFuncSetAttribute(select_radix, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxStagedKeys * (int)sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(kClusterCtas, d.Hkv, d.B);
+  select_radix<<<grid, kThreads, smem, st>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kept, int32_t* perm,
@@ -371,10 +399,7 @@ cudaError_t launch_select(const Dims& d, const float* scores, const Budgets& kep
   a.mass_scale = 0.f;
   a.k_out = nullptr;
   a.kept = kept;
-  const dim3 grid(kClusterCtas, d.Hkv, d.B);
-  select_radix<<<grid, kThreads, 0, st>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_radix(d, a, st);
 }
 
 cudaError_t launch_select_coverage(const Dims& d, const float* scores, double tau, int32_t* perm, int32_t* k_out,
@@ -392,10 +417,7 @@ cudaError_t launch_select_coverage(const Dims& d, const float* scores, double ta
   a.mass_scale = ldexpf(1.f, 55 - lg);
   a.k_out = k_out;
   for (int i = 0; i < kMaxGroups; ++i) a.kept.kept[i] = 0;
-  const dim3 grid(kClusterCtas, d.Hkv, d.B);
-  select_radix<<<grid, kThreads, 0, st>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_radix(d, a, st);
 }
 
 }  // namespace tsa
