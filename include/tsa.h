@@ -183,10 +183,10 @@ TSA_API tsa_status tsa_zero_dropped(const tsa_desc* desc, const int32_t* perm, c
  * array built into the library, reserved on every GPU that loads it until the
  * process exits.  Checks run in this order: the shape (as tsa_score), then
  * the partials' size -- B*Hkv * splits * rows * 8 bytes above 1 MiB returns
- * TSA_ERR_WORKSPACE, with splits = min(ceil(L/128), 37) and rows = 128 or 256
+ * TSA_ERR_WORKSPACE, with splits = min(ceil(L/128), 18) and rows = 128 or 256
  * (G*window <= 128 or not) in bf16, splits = min(ceil(L/64), 74) and rows =
  * G*window rounded up to 64 in f32; the 32/8-head, window-64 layer fits at
- * B = 1 up to L = 131072 in bf16 (606 KB) and up to B = 64 at L <= 128 --
+ * B = 1 up to L = 131072 in bf16 (295 KB) and up to B = 64 at L <= 128 --
  * then the pointers (TSA_ERR_INVALID_ARG).  The first call made
  * with a device current looks up the array's device address; make that first
  * call before any stream capture.  All calls share the array: calls whose

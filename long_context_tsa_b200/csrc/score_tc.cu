@@ -506,13 +506,13 @@ cudaError_t launch_passes(const Dims& d, const CUtensorMap& mq, const CUtensorMa
 
 }  // namespace
 
-// Key-range splits per KV head: a function of L only (at most 37, so 8 KV heads
-// make exactly two waves of one CTA per SM on 148 SMs).  A KV head's scores
-// therefore do not depend on which other heads share the call: a layer split by
-// KV group across calls (or GPUs) gives bit-identical scores.
+// Key-range splits per KV head: a function of L only (at most 18, so a layer of
+// 8 KV heads is one wave of 144 CTAs, one per SM).  A KV head's scores therefore
+// do not depend on which other heads share the call: a layer split by KV group
+// across calls (or GPUs) gives bit-identical scores.
 int score_tc_splits(const Dims& d) {
   const int ntiles = (d.L + 127) / 128;
-  const int s = ntiles < 37 ? ntiles : 37;
+  const int s = ntiles < 18 ? ntiles : 18;
   return s < kMaxScoreSplits ? s : kMaxScoreSplits;
 }
 

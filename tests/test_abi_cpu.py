@@ -162,7 +162,7 @@ def test_zero_dropped_and_noalloc_reject_before_launch(lib):
         assert lib.tsa_score_noalloc(ctypes.byref(fits), None, None, 64, None, None) == inv
         two_splits = N.make_desc(B=64, Hq=32, Hkv=8, L=2 * L_fit, D=128, dtype=dt)
         assert lib.tsa_score_noalloc(ctypes.byref(two_splits), None, None, 64, None, None) == wsz
-    # The bf16 128K layer (8 KV heads x 37 splits x 256 rows x 8 bytes = 606 KB) fits.
+    # The bf16 128K layer (8 KV heads x 18 splits x 256 rows x 8 bytes = 295 KB) fits.
     layer = N.make_desc(B=1, Hq=32, Hkv=8, L=131072, D=128, dtype=N.TSA_BF16)
     assert lib.tsa_score_noalloc(ctypes.byref(layer), None, None, 64, None, None) == inv
     assert lib.tsa_score_noalloc(ctypes.byref(desc(D=96)), None, None, 64, None, None) == \

@@ -79,7 +79,7 @@ def test_noalloc_score_fills_the_whole_array_at_its_limit():
 
 
 def test_noalloc_score_bench_layer():
-    # The 128K bf16 layer (8 KV heads x 37 splits x 256 rows x 8 bytes = 606 KB) fits.
+    # The 128K bf16 layer (8 KV heads x 18 splits x 256 rows x 8 bytes = 295 KB) fits.
     w = I.WORKLOADS["gqa_bf16_L131072"]
     _check(w, seed=4, with_oracle=False)
 
