@@ -14,12 +14,15 @@
 //           c_r = m_r + log2 Z_r combined over all splits,
 //           score[j] = sum_r 2^(x_rj - c_r)  -- one thread per key, no
 //           cross-thread reduction.
-// Warp roles (576 threads): warps 0-15 read TMEM (four warpgroups; each
-// thread takes half of its TMEM row's columns, so every SM sub-partition has
-// four reader warps to hide the exponential unit's latency), warp 16 loads
-// (TMA), warp 17 issues tcgen05.mma.  Pass 1 merges the two column halves of
-// each row's (m, Z); pass 2 adds the two halves of each key's sum into the
-// scores, which pass 1 zeroed.  Bounded waits throughout.
+// Warp roles (576 threads): warps 0-15 read TMEM (four warpgroups), warp 16
+// loads (TMA), warp 17 issues tcgen05.mma.  Two TMEM buffers alternate by step;
+// in pass 1 each warpgroup pair reads every other step (whole rows), in pass 2
+// each warpgroup pair reads every other key tile (one column half each), so on
+// every SM sub-partition two reader warps load from TMEM while the other two
+// compute.  TMEM loads run one 32-column chunk ahead.  Pass 1 merges the
+// partial (m, Z) of the two step parities of each row; pass 2 adds the two
+// halves of each key's sum into the scores, which pass 1 zeroed.  Bounded
+// waits throughout.
 #include <cuda.h>
 #include <math.h>
 
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_sfull(i), 1);
-      mbar_init(bar_sfree(i), PASS == 1 ? kReaders : kReaders / 2);
+      mbar_init(bar_sfree(i), kReaders / 2);  // one warpgroup pair reads each buffer
     }
     mbar_init(bar_td, 1);
     *abort_flag = 0;
@@ -285,101 +288,109 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ TMEM readers
     const int wg = warp >> 2;       // 0..3
-    const int a = wg & 1;           // row half (pass 1, RH == 2) or tile parity
-    const int ch = wg >> 1;         // column half of the TMEM row this thread reads
+    const int a = wg & 1;           // pass 1: row block (RH == 2) or tile of the step (RH == 1); pass 2: tile parity
+    const int pr = wg >> 1;         // pass 1: step parity this pair reads; pass 2: column half
+    const int ch = pr;
     const int rl = threadIdx.x & 127;  // TMEM lane of this thread
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
     if (PASS == 1) {
+      // The two warpgroup pairs take alternate steps (buffer bf = step parity), so
+      // one pair's TMEM loads overlap the other pair's exponentials; a thread reads
+      // all 128 columns of its row in 32-column chunks, one chunk loaded ahead.
       const int r = RH == 2 ? a * 128 + rl : rl;  // window row
       const int pos = L - p.W + (r % p.W);
       const bool row_ok = r < p.M;
       // Pass 2 adds its two column halves into the scores: start them at zero.
       for (int j = j0 + threadIdx.x; j < j1; j += kReaders) p.scores[(size_t)grp * L + j] = 0.f;
       float m = -INFINITY, z = 0.f;
-      for (int i = 0; i < nstep; ++i) {
-        const int bf = i & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (i >> 1) & 1, p.wait_limit, abort_flag));
+      // z is kept relative to a per-row reference m: any reference gives the
+      // same m + log2 z.  The first chunk with a visible key sets m to its exact
+      // max; later chunks sum 2^(x - m) directly and are redone against their own
+      // max only if the sum leaves a safe range (a key far above m).
+      auto chunk_sum = [&](const uint32_t (&v)[32], float ref) {
+        const uint64_t negm2 = f2_pack(-ref, -ref), sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, negm2), t0, t1);
+          float p0, p1;
+          if (e2 % 3 == 2) {  // one pair in three on the FMA pipe; t <= 127 there (clamped: a
+                              // larger t saturates at 2^127 and the sum check below redoes the chunk)
+            ex2_fma_pair(fminf(t0, 127.f), fminf(t1, 127.f), p0, p1);
+          } else {
+            p0 = ex2_approx(t0);
+            p1 = ex2_approx(t1);
+          }
+          a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(p0, p1));
+        }
+        float s0, s1, s2, s3, s4, s5, s6, s7;
+        f2_unpack(a2[0], s0, s1);
+        f2_unpack(a2[1], s2, s3);
+        f2_unpack(a2[2], s4, s5);
+        f2_unpack(a2[3], s6, s7);
+        return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+      };
+      for (int i = pr; i < nstep; i += 2) {
+        const int bf = i & 1;  // == pr
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(bar_sfull(bf), (i >> 1) & 1, p.wait_limit, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        const int u = RH == 2 ? i : 2 * i + a;
-        uint32_t v[64];
-        if (u < nt) {
-          const uint32_t ta = tmem + lane_off + bf * 256 + a * 128 + ch * 64;
-          tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_wait_ld32(*reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_wait_ld32(*reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        }
-        tc_fence_before();
-        mbar_arrive(bar_sfree(bf));
-        if (u < nt) {
-          const int kbase = j0 + 128 * u + 64 * ch;
-          const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this half tile
-          const bool masked = __any_sync(0xffffffffu, lim < 64);
-          if (masked) {
+        const int u = RH == 2 ? i : 2 * i + a;  // key tile of this thread's row
+        const bool have = u < nt;
+        const uint32_t ta = tmem + lane_off + bf * 256 + a * 128;
+        uint32_t va[32], vb[32];
+        if (have) tmem_ld32(ta, va);
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (e >= lim) v[e] = 0xff800000u;  // -inf
+        for (int q = 0; q < 4; ++q) {
+          uint32_t(&v)[32] = (q & 1) ? vb : va;
+          uint32_t(&vn)[32] = (q & 1) ? va : vb;
+          if (have && q < 3) tmem_ld32_async(ta + (q + 1) * 32, vn);
+          if (q == 3) {  // every column of this buffer is in registers: release it
+            tc_fence_before();
+            mbar_arrive(bar_sfree(bf));
           }
-          // z is kept relative to a per-row reference m: any reference gives the
-          // same m + log2 z.  The first tile with a visible key sets m to its exact
-          // max; later tiles sum 2^(x - m) directly and are redone against their own
-          // max only if the sum leaves a safe range (a key far above m).
-          auto tile_sum = [&](float ref) {
-            const uint64_t negm2 = f2_pack(-ref, -ref), sc2 = f2_pack(p.scale_log2, p.scale_log2);
-            uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
+          if (have) {
+            const int kbase = j0 + 128 * u + 32 * q;
+            const int lim = row_ok ? min(j1 - 1, pos) - kbase + 1 : 0;  // visible keys in this chunk
+            if (__any_sync(0xffffffffu, lim < 32)) {
 #pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) {
-              float t0, t1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), sc2, negm2), t0, t1);
-              float p0, p1;
-              if (e2 % 3 == 2) {  // one pair in three on the FMA pipe; t <= 127 there (clamped: a
-                                  // larger t saturates at 2^127 and the sum check below redoes the tile)
-                ex2_fma_pair(fminf(t0, 127.f), fminf(t1, 127.f), p0, p1);
-              } else {
-                p0 = ex2_approx(t0);
-                p1 = ex2_approx(t1);
+              for (int e = 0; e < 32; ++e)
+                if (e >= lim) v[e] = 0xff800000u;  // -inf
+            }
+            float st = (m > -INFINITY) ? chunk_sum(v, m) : INFINITY;
+            const bool exact = !(st <= 1.8446744e19f);  // > 2^64, NaN, or no reference yet
+            if (__any_sync(0xffffffffu, exact)) {
+              float mx8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
+#pragma unroll
+              for (int e = 8; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+              const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
+              if (exact && mt > -INFINITY) {
+                const float mn = fmaxf(m, mt);
+                const float zs = (m > -INFINITY) ? z * ex2_approx(m - mn) : 0.f;
+                m = mn;
+                z = zs;
               }
-              a2[e2 & 3] = f2_add(a2[e2 & 3], f2_pack(p0, p1));
+              if (exact) st = (m > -INFINITY) ? chunk_sum(v, m) : 0.f;
             }
-            float s0, s1, s2, s3, s4, s5, s6, s7;
-            f2_unpack(a2[0], s0, s1);
-            f2_unpack(a2[1], s2, s3);
-            f2_unpack(a2[2], s4, s5);
-            f2_unpack(a2[3], s6, s7);
-            return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-          };
-          float st = (m > -INFINITY) ? tile_sum(m) : INFINITY;
-          const bool exact = !(st <= 1.8446744e19f);  // > 2^64, NaN, or no reference yet
-          if (__any_sync(0xffffffffu, exact)) {
-            float mx8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(v[e]);
-#pragma unroll
-            for (int e = 8; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-            const float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
-            if (exact && mt > -INFINITY) {
-              const float mn = fmaxf(m, mt);
-              const float zs = (m > -INFINITY) ? z * ex2_approx(m - mn) : 0.f;
-              m = mn;
-              z = zs;
-            }
-            if (exact) st = (m > -INFINITY) ? tile_sum(m) : 0.f;
+            z += st;
           }
-          z += st;
+          if (have && q < 3) tmem_wait_ld32(vn);
         }
       }
       // Merge the partial (m, Z) of the warpgroups that saw the same rows: both
-      // column halves, and for RH == 1 also both tile parities.  The named
+      // step parities, and for RH == 1 also both tiles of a step.  The named
       // barrier is reached by all reader threads whatever happened above.
-      const int slot = RH == 2 ? (ch * 2 + a) : wg;  // 4 slots of 128 (RH == 1) or 2 x 2 (RH == 2)
+      const int slot = RH == 2 ? (pr * 2 + a) : wg;  // 4 slots of 128 (RH == 1) or 2 x 2 (RH == 2)
       red[slot * 128 + rl] = m;
       red[512 + slot * 128 + rl] = z;
       asm volatile("bar.sync 1, %0;" ::"n"(kReaders) : "memory");
       if (!ok) fail();
-      const bool writer = RH == 2 ? (ch == 0) : (wg == 0);
+      const bool writer = RH == 2 ? (pr == 0) : (wg == 0);
       if (writer && !*abort_flag) {
         constexpr int NSRC = RH == 2 ? 2 : 4;  // partials per row
         float ms[NSRC], zs4[NSRC];
@@ -430,11 +441,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (TMEM loads are warp-collective).
         const bool tail = __any_sync(0xffffffffu, key >= L - p.W);
         float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+        // 32-column chunks with the next chunk's TMEM load in flight; the buffer
+        // is released once its last chunk is in registers.
+        const uint32_t tb = tmem + lane_off + bf * 256 + ch * HC;
+        uint32_t va[32], vb[32];
+        tmem_ld32(tb, va);
+#pragma unroll
         for (int q4 = 0; q4 < HC / 32; ++q4) {
           const int col0 = ch * HC + q4 * 32;  // first window row of this chunk
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + bf * 256 + col0, v);
+          uint32_t(&v)[32] = (q4 & 1) ? vb : va;
+          uint32_t(&vn)[32] = (q4 & 1) ? va : vb;
+          if (q4 + 1 < HC / 32) {
+            tmem_ld32_async(tb + (q4 + 1) * 32, vn);
+          } else {
+            tc_fence_before();
+            mbar_arrive(bar_sfree(bf));
+          }
           const float* nc = cst + col0;
           if (!tail) {
             const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
@@ -468,10 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc4[e & 3] += (key > L - p.W + (col % p.W)) ? 0.f : pe;
             }
           }
+          if (q4 + 1 < HC / 32) tmem_wait_ld32(vn);
         }
         const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-        tc_fence_before();
-        mbar_arrive(bar_sfree(bf));
         // Two column halves per key: 0 + h0 + h1 is the same in either order.
         if (key < j1) atomicAdd(out + key, acc);
       }
