@@ -328,6 +328,13 @@ TSA_API const char* tsa_status_string(tsa_status s);
 TSA_API void tsa_debug_set_wait_limit(uint64_t polls);
 /* Number of kernels this library has launched in this process (all devices). */
 TSA_API uint64_t tsa_debug_launch_count(void);
+/* Number of those that were the two-SM attention kernel (d = 128 on CTA pairs,
+ * cta_group::2), which tsa_attend, tsa_attend_accumulate,
+ * tsa_attend_block_sparse and the forward calls use in place of the one-SM
+ * kernel while the environment variable TSA_ATTEND_CTA_PAIRS is set to a
+ * value other than "0" (read at every launch; same arguments and results
+ * within the attention tolerance; off by default). */
+TSA_API uint64_t tsa_debug_cta_pair_launch_count(void);
 TSA_API tsa_status tsa_debug_wait_never_set(void* ws, size_t ws_bytes, void* stream);
 /* y = 2^x through the FMA-pipe exponential the scoring kernel uses for one
  * pair of values in three (device arrays of n floats, n even, 16-byte aligned). */

@@ -22,6 +22,7 @@ from ._native import (  # noqa: F401
     tsa_check_status,
     tsa_debug_exp2,
     tsa_debug_launch_count,
+    tsa_debug_cta_pair_launch_count,
     tsa_debug_set_wait_limit,
     tsa_debug_wait_never_set,
     tsa_drift,

@@ -22,7 +22,7 @@ STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
 EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select", "tsa_attend", "tsa_forward",
             "tsa_forward_host", "tsa_check_status", "tsa_status_string", "tsa_debug_set_wait_limit",
-            "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_score_noalloc",
+            "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_debug_cta_pair_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
             "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2", "tsa_zero_dropped",
             "tsa_out_proj_workspace_size", "tsa_out_proj")
@@ -57,6 +57,7 @@ _SIGS = {
     "tsa_debug_set_wait_limit": (None, [ctypes.c_uint64]),
     "tsa_debug_wait_never_set": (ctypes.c_int, [_P, _SZ, _P]),
     "tsa_debug_launch_count": (ctypes.c_uint64, []),
+    "tsa_debug_cta_pair_launch_count": (ctypes.c_uint64, []),
     "tsa_score_noalloc": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _I32, _P, _P]),
     "tsa_attend_accumulate": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_drift_workspace_size": (_SZ, []),
@@ -227,6 +228,11 @@ def tsa_debug_wait_never_set(ws, stream=None):
 def tsa_debug_launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(lib().tsa_debug_launch_count())
+
+
+def tsa_debug_cta_pair_launch_count() -> int:
+    """Launches of the two-SM attention kernel (opt-in: TSA_ATTEND_CTA_PAIRS=1) so far in this process."""
+    return int(lib().tsa_debug_cta_pair_launch_count())
 
 
 def tsa_score_noalloc(desc, q, k, window, scores, stream=None):

@@ -37,6 +37,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <type_traits>
 
 #include "device_common.cuh"
@@ -568,8 +570,14 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
                              const Budgets& kept, void* out, uint32_t* status, bool accumulate,
                              const uint8_t* block_mask, cudaStream_t st) {
-  return d.D == 64 ? launch_tc<64>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st)
-                   : launch_tc<128>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st);
+  if (d.D == 64) return launch_tc<64>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st);
+  // The two-SM form (attend_tc2.cu) is opt-in: it measured slower than this
+  // kernel at every bench size (the per-tile softmax chain, not the loads or
+  // the MMA rate, bounds both).
+  const char* pairs = getenv("TSA_ATTEND_CTA_PAIRS");
+  if (pairs != nullptr && pairs[0] != '\0' && strcmp(pairs, "0") != 0)
+    return launch_attend_tc_pair(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st);
+  return launch_tc<128>(d, q, k, v, perm, kept, out, status, accumulate, block_mask, st);
 }
 
 }  // namespace tsa

@@ -45,6 +45,7 @@ int window_rows_padded(const Dims& d, int window);  // Mp: G*window rounded up t
 
 uint64_t wait_limit();  // polls for device bounded waits
 void count_launches(int n);  // every launcher reports the kernels it enqueued
+void count_pair_launch();    // the two-SM attention kernel reports each launch here too
 
 // Kept counts clamped to L, one per (b, g); filled by the host entry points.
 struct Budgets {
@@ -69,6 +70,10 @@ cudaError_t launch_attend_simt(const Dims& d, const void* q, const void* k, cons
 cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
                              const Budgets& kept, void* out, uint32_t* status, bool accumulate,
                              const uint8_t* block_mask, cudaStream_t st);
+// d = 128 on CTA pairs (cta_group::2): the same operation as launch_attend_tc.
+cudaError_t launch_attend_tc_pair(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
+                                  const Budgets& kept, void* out, uint32_t* status, bool accumulate,
+                                  const uint8_t* block_mask, cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
 // Output projection (out_proj.cu): its own workspace, a 256-byte status header

@@ -20,6 +20,10 @@ static std::atomic<uint64_t> g_launches{0};
 
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+static std::atomic<uint64_t> g_pair_launches{0};
+
+void count_pair_launch() { g_pair_launches.fetch_add(1, std::memory_order_relaxed); }
+
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int window_rows_padded(const Dims& d, int window) {
@@ -435,6 +439,8 @@ const char* tsa_status_string(tsa_status s) {
 void tsa_debug_set_wait_limit(uint64_t polls) { g_wait_limit.store(polls, std::memory_order_relaxed); }
 
 uint64_t tsa_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint64_t tsa_debug_cta_pair_launch_count(void) { return g_pair_launches.load(std::memory_order_relaxed); }
 
 tsa_status tsa_debug_exp2(const float* x, float* y, int32_t n, void* stream) {
   if (!aligned16(x) || !aligned16(y) || n < 2 || (n & 1)) return TSA_ERR_INVALID_ARG;
