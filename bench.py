@@ -84,6 +84,11 @@ def block_sparse_flops(w, budgets, bm) -> float:
     return total
 
 
+# Share of the score's exponentials that run on the exponential unit: in every
+# 16-pair chunk, pairs 2, 5, 8, 11 and 14 use the FMA-pipe polynomial instead.
+SCORE_MUFU_SHARE = 11.0 / 16.0
+
+
 def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: str):
     """The step's other kernels against their own bounds.
 
@@ -109,7 +114,10 @@ def other_rooflines(w, t_score_ms: float, t_select_ms: float, peaks, peak_src: s
         {"kernel": "score_tc (2 passes)", "bound": "alu", "achieved": a_score / 1e12, "peak": mufu_peak / 1e12,
          "unit": "Tex2/s", "frac": a_score / mufu_peak,
          "peak_source": f"16 ex2/clk/SM x {sms} SMs x {mhz:.0f} MHz (max SM clock)",
-         "note": "one exponential pair in three runs on the FMA pipe, so this is an effective rate"},
+         "mufu_share": SCORE_MUFU_SHARE, "mufu_issued_achieved": a_score * SCORE_MUFU_SHARE / 1e12,
+         "mufu_issued_frac": a_score * SCORE_MUFU_SHARE / mufu_peak,
+         "note": "achieved/frac count every exponential (an effective rate: 5 pairs in 16 run on the FMA "
+                 "pipe); mufu_issued_* count only those the exponential unit executes"},
         {"kernel": "score_tc (2 passes)", "bound": "hbm", "achieved": a_sc_hbm, "peak": hbm, "unit": "GB/s",
          "frac": a_sc_hbm / hbm, "peak_source": f"hbm_gbs ({peak_src})",
          "note": "algorithmic bytes (K once, window queries, scores); the exponentials bound it first"},

@@ -1,6 +1,8 @@
 """Host-side helpers of bench.py: the flop and byte counts behind the reported
 rooflines (no GPU needed)."""
 
+import os
+
 import numpy as np
 
 import bench
@@ -49,6 +51,12 @@ def test_other_rooflines_counts():
     # 2 passes x (B x Hkv) groups x (G x W) window rows x L keys exponentials
     assert abs(score["achieved"] * 1e12 * 0.19e-3 - 2 * 8 * 4 * 64 * 131072) < 1e3
     assert score["bound"] == "alu" and 0 < score["frac"] < 1
+    # Only the exponentials the MUFU executes: the share matches the kernel's split
+    # (in both passes, pair e2 of each 16-pair chunk goes to the FMA pipe when e2 % 3 == 2).
+    src = open(os.path.join(os.path.dirname(bench.__file__), "long_context_tsa_b200", "csrc", "score_tc.cu")).read()
+    assert src.count("if (e2 % 3 == 2) {") == 2
+    assert score["mufu_share"] == sum(1 for e2 in range(16) if e2 % 3 != 2) / 16
+    assert abs(score["mufu_issued_frac"] - score["frac"] * score["mufu_share"]) < 1e-12
     # scores read once and the permutation written once: 8 bytes per key per group
     assert abs(select["achieved"] * 1e9 * 0.031e-3 - 8 * 8 * 131072) < 1.0
     assert select["bound"] == "hbm" and 0 < select["frac"] < 1
