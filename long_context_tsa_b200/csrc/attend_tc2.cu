@@ -17,9 +17,15 @@
 // value dims (all 128 keys) -- so each CTA gathers half of every K and V tile.
 // CTA 0 (leader) issues the MMAs and commits every completion to both CTAs'
 // barriers; CTA 1's MMA warp relays its producers' cp.async completions to the
-// leader's barriers; both CTAs' softmax warps tell the leader that P is in TMEM
-// with one cluster-scope arrive per warp.  Warp roles, TMEM columns, the online
-// softmax, the scatter epilogue and the fused zero fill are attend_tc's.
+// leader's barriers (async-proxy fence, then a cluster-scope release arrive);
+// the softmax warps tell the leader that P is in TMEM with one arrive per warp
+// on the leader's barrier (a local arrive in CTA 0, the CTA-scope remote arrive
+// in CTA 1: the TMEM stores were already waited for and fenced, and a
+// cluster-scope release there costs about a thousand cycles per step).  Warp
+// roles, TMEM columns, the online softmax, the scatter epilogue and the fused
+// zero fill are attend_tc's.  The library runs this kernel only on request
+// (TSA_ATTEND_CTA_PAIRS): it measured slower than attend_tc, whose bound (the
+// per-tile softmax-to-MMA chain) it shares.
 // Every mbarrier wait is bounded; on timeout a CTA records TSA_ERR_TIMEOUT,
 // drains its own copies and MMAs, meets its peer at the final cluster barrier,
 // frees TMEM and exits.
