@@ -38,7 +38,7 @@ namespace {
 
 constexpr int kClusterCtas = 8;
 constexpr int kThreads = 1024;
-constexpr int kPerThread = 4;
+constexpr int kPerThread = 8;
 constexpr int kChunk = kThreads * kPerThread;
 // A CTA's slice of sortable keys is staged in shared memory once when it holds
 // at most this many (160 KB): every radix pass, the counts and the compaction
@@ -324,7 +324,14 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads,
     gt_before = (uint32_t)lo;  // everything is kept: index i lands at i
   }
 
+  // A chunk's kept indices land in one contiguous range of perm[0:K] and its
+  // dropped ones in one contiguous range of perm[K:L]: each index goes to its
+  // place in a shared-memory copy of the chunk's two ranges (kept first), and
+  // the ranges are then written out with consecutive threads on consecutive
+  // addresses.
+  __shared__ int32_t stage[kChunk];
   for (int base = lo; base < hi; base += kChunk) {
+    const int n = min(kChunk, hi - base);
     const int i0 = base + tid * kPerThread;
     uint32_t isgt[kPerThread], iseq[kPerThread];
     uint32_t ngt = 0u, neq = 0u;
@@ -347,6 +354,9 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads,
     }
     uint32_t total;
     const uint32_t ex = block_exclusive_scan((neq << 16) | ngt, warp_sums, total);
+    const uint32_t tg = total & 0xFFFFu, te = total >> 16;
+    const uint32_t kb0 = gt_before + min(eq_before, krem);            // kept indices before the chunk
+    const uint32_t nk = gt_before + tg + min(eq_before + te, krem) - kb0;  // kept indices in the chunk
     uint32_t gb = gt_before + (ex & 0xFFFFu);
     uint32_t eb = eq_before + (ex >> 16);
 #pragma unroll
@@ -355,9 +365,10 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads,
       if (i < hi) {
         const uint32_t S = gb + min(eb, krem);  // kept indices before i
         const bool keep = isgt[e] || (iseq[e] && eb < krem);
-        const uint32_t dst = keep ? S : (uint32_t)K + (uint32_t)i - S;
-        if (dst < (uint32_t)L) {
-          pm[dst] = i;
+        // kept: S - kb0 in [0, nk); dropped: i - S dropped before i, minus those before the chunk
+        const uint32_t local = keep ? S - kb0 : nk + ((uint32_t)i - S) - ((uint32_t)base - kb0);
+        if (local < (uint32_t)n) {
+          stage[local] = i;
         } else {
           record_status(a.status, TSA_ERR_DEVICE_BOUNDS);
         }
@@ -365,8 +376,18 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads,
         eb += iseq[e];
       }
     }
-    gt_before += total & 0xFFFFu;
-    eq_before += total >> 16;
+    __syncthreads();
+    for (int x = tid; x < n; x += kThreads) {
+      const uint32_t dst = (uint32_t)x < nk ? kb0 + (uint32_t)x : (uint32_t)K + ((uint32_t)base - kb0) + ((uint32_t)x - nk);
+      if (dst < (uint32_t)L) {
+        pm[dst] = stage[x];
+      } else {
+        record_status(a.status, TSA_ERR_DEVICE_BOUNDS);
+      }
+    }
+    __syncthreads();  // the stage is rewritten by the next chunk
+    gt_before += tg;
+    eq_before += te;
   }
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
