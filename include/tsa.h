@@ -265,17 +265,34 @@ TSA_API tsa_status tsa_forward_coverage(const tsa_desc* desc, const void* q, con
                                         size_t ws_bytes, void* stream);
 
 /*
- * tsa_forward_host -- tsa_forward on HOST inputs and output.  q_host/k_host/
- * v_host are copied into the caller's device buffers q_dev/k_dev/v_dev with
- * one cudaMemcpyAsync each, the forward runs, and out_dev is copied back to
- * out_host; all on `stream`.  The call returns after enqueueing; the host
- * buffers must stay valid (and should be pinned for asynchrony) until the
- * stream reaches that point.
+ * tsa_forward_host -- tsa_forward on HOST inputs and output, all on `stream`;
+ * out_dev is copied back to out_host in full.  The inputs reach the caller's
+ * device buffers q_dev/k_dev/v_dev in one of two ways:
+ * - q_host and v_host both mapped into the device's address space (pinned
+ *   with the mapped flag; cudaHostAlloc memory is mapped under unified
+ *   addressing): only what the step reads crosses the host link ([P1] Step 2
+ *   gathers only the selected tokens; [P2] Figure 3, Stage 1).  K is copied
+ *   in full (every key is scored), and the last `window` rows of every query
+ *   head are copied.  After the selection a kernel reads the kept rows of Q
+ *   (the G heads of each KV group) and of V in place and writes them to the
+ *   same positions of q_dev / v_dev.  Other rows of q_dev / v_dev are not
+ *   written.
+ * - otherwise: one cudaMemcpyAsync of each whole input, then tsa_forward.
+ * The result in out_host is the same either way.  The call returns after
+ * enqueueing; the host buffers must stay valid until the stream reaches that
+ * point.  TSA_ERR_DEVICE_BOUNDS (status word) for a permutation entry
+ * outside [0, L).
  */
 TSA_API tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void* k_host,
                             const void* v_host, int32_t window, const int32_t* budget_host,
                             void* out_host, void* q_dev, void* k_dev, void* v_dev, void* out_dev,
                             void* ws, size_t ws_bytes, void* stream);
+/* Host-to-device bytes tsa_forward_host moves for these arguments: K in full,
+ * plus either the window rows of Q and the kept rows of Q (G per kept
+ * position) and of V (mapped q_host and v_host), or all of Q and V.  0 for an
+ * invalid shape, window or budget. */
+TSA_API size_t tsa_forward_host_h2d_bytes(const tsa_desc* desc, int32_t window, const int32_t* budget_host,
+                                          const void* q_host, const void* v_host);
 
 /*
  * tsa_drift -- representation drift between two hidden-state tensors

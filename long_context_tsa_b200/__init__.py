@@ -30,6 +30,7 @@ from ._native import (  # noqa: F401
     tsa_forward,
     tsa_forward_coverage,
     tsa_forward_host,
+    tsa_forward_host_h2d_bytes,
     tsa_layer_stable,
     tsa_out_proj,
     tsa_out_proj_workspace_size,

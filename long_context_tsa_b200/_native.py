@@ -25,7 +25,7 @@ EXPORTED = ("tsa_workspace_size", "tsa_workspace_init", "tsa_score", "tsa_select
             "tsa_debug_wait_never_set", "tsa_debug_launch_count", "tsa_debug_cta_pair_launch_count", "tsa_score_noalloc",
             "tsa_attend_accumulate", "tsa_drift_workspace_size", "tsa_drift", "tsa_layer_stable",
             "tsa_select_coverage", "tsa_forward_coverage", "tsa_attend_block_sparse", "tsa_debug_exp2", "tsa_zero_dropped",
-            "tsa_out_proj_workspace_size", "tsa_out_proj")
+            "tsa_out_proj_workspace_size", "tsa_out_proj", "tsa_forward_host_h2d_bytes")
 
 
 class TsaDesc(ctypes.Structure):
@@ -52,6 +52,7 @@ _SIGS = {
     "tsa_forward": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "tsa_forward_host": (ctypes.c_int, [ctypes.POINTER(TsaDesc), _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _P,
                                         _SZ, _P]),
+    "tsa_forward_host_h2d_bytes": (_SZ, [ctypes.POINTER(TsaDesc), _I32, _P, _P, _P]),
     "tsa_check_status": (ctypes.c_int, [_P, _SZ, _P]),
     "tsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "tsa_debug_set_wait_limit": (None, [ctypes.c_uint64]),
@@ -198,6 +199,12 @@ def tsa_forward_host(desc, q_host, k_host, v_host, window, budgets, out_host, q_
     _check(lib().tsa_forward_host(ctypes.byref(desc), _ptr(q_host), _ptr(k_host), _ptr(v_host), int(window),
                                   _budgets(budgets), _ptr(out_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
                                   _ptr(out_dev), _ptr(ws), ws.numel(), _stream(stream)), "tsa_forward_host")
+
+
+def tsa_forward_host_h2d_bytes(desc, window, budgets, q_host, v_host) -> int:
+    """Host-to-device bytes ``tsa_forward_host`` moves for these host inputs (0 for invalid arguments)."""
+    return int(lib().tsa_forward_host_h2d_bytes(ctypes.byref(desc), int(window), _budgets(budgets), _ptr(q_host),
+                                                _ptr(v_host)))
 
 
 def tsa_check_status(ws, stream=None) -> int:

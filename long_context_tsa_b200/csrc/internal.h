@@ -74,6 +74,12 @@ cudaError_t launch_attend_tc(const Dims& d, const void* q, const void* k, const 
 cudaError_t launch_attend_tc_pair(const Dims& d, const void* q, const void* k, const void* v, const int32_t* perm,
                                   const Budgets& kept, void* out, uint32_t* status, bool accumulate,
                                   const uint8_t* block_mask, cudaStream_t st);
+// Kept rows of Q (the G query heads of each group) and V, read from host
+// memory mapped into the device address space, written to the same positions
+// of the device buffers (host_gather.cu).
+cudaError_t launch_gather_kept_rows(const Dims& d, const void* q_src, const void* v_src, const int32_t* perm,
+                                    const Budgets& kept, void* q_dst, void* v_dst, uint32_t* status,
+                                    cudaStream_t st);
 cudaError_t launch_zero_fill(const Dims& d, const int32_t* perm, const Budgets& kept, void* out,
                              uint32_t* status, cudaStream_t st);
 // Output projection (out_proj.cu): its own workspace, a 256-byte status header

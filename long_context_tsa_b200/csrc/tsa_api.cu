@@ -374,6 +374,33 @@ tsa_status tsa_forward_coverage(const tsa_desc* desc, const void* q, const void*
   return run_attend(d, q, k, v, perm, kb, out, ws, st);
 }
 
+namespace {
+
+// The device address of host memory that is mapped into this device's address
+// space (pinned with the mapped flag, implied for cudaHostAlloc under unified
+// addressing), or null for pageable memory.
+const void* mapped_device_ptr(const void* host) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+// Host-to-device bytes of tsa_forward_host; sparse: q and v are read in place.
+size_t host_h2d_bytes(const Dims& d, int window, const Budgets& kb, bool sparse) {
+  const size_t esz = d.dtype == TSA_F32 ? 4 : 2;
+  const size_t row = (size_t)d.D * esz;
+  const size_t kvbytes = (size_t)d.B * d.Hkv * d.L * row;
+  if (!sparse) return (size_t)d.B * d.Hq * d.L * row + 2 * kvbytes;
+  size_t kept = 0;
+  for (int i = 0; i < d.B * d.Hkv; ++i) kept += (size_t)kb.kept[i];
+  return kvbytes + (size_t)d.B * d.Hq * window * row + kept * (size_t)(d.G + 1) * row;
+}
+
+}  // namespace
+
 tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void* k_host, const void* v_host,
                             int32_t window, const int32_t* budget_host, void* out_host, void* q_dev, void* k_dev,
                             void* v_dev, void* out_dev, void* ws, size_t ws_bytes, void* stream) {
@@ -387,16 +414,53 @@ tsa_status tsa_forward_host(const tsa_desc* desc, const void* q_host, const void
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(out_dev)) return TSA_ERR_INVALID_ARG;
   if ((s = check_window(d, window)) != TSA_OK) return s;
-  if (ws_bytes < ws_layout(d, window).total) return TSA_ERR_WORKSPACE;
+  const WsLayout w = ws_layout(d, window);
+  if (ws_bytes < w.total) return TSA_ERR_WORKSPACE;
   Budgets kb;
   if ((s = load_budgets(d, budget_host, &kb)) != TSA_OK) return s;
-  if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
-  if (cudaMemcpyAsync(k_dev, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
-  if (cudaMemcpyAsync(v_dev, v_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
-  s = tsa_forward(desc, q_dev, k_dev, v_dev, window, budget_host, nullptr, nullptr, out_dev, ws, ws_bytes, stream);
-  if (s != TSA_OK) return s;
+  const void* q_map = mapped_device_ptr(q_host);
+  const void* v_map = mapped_device_ptr(v_host);
+  if (q_map == nullptr || v_map == nullptr || !aligned16(q_map) || !aligned16(v_map)) {
+    // Full copies of the three inputs, then the device forward.
+    if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+    if (cudaMemcpyAsync(k_dev, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+    if (cudaMemcpyAsync(v_dev, v_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+    s = tsa_forward(desc, q_dev, k_dev, v_dev, window, budget_host, nullptr, nullptr, out_dev, ws, ws_bytes, stream);
+    if (s != TSA_OK) return s;
+  } else {
+    // Mapped q and v: only what the step reads crosses the host link.  Every
+    // key is scored, so K is copied in full; the score's queries are the last
+    // `window` rows of each head (one strided copy); after the selection the
+    // gather kernel reads the kept rows of Q and V in place.
+    if (cudaMemcpyAsync(k_dev, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return TSA_ERR_CUDA;
+    const size_t pitch = (size_t)d.L * d.D * esz, wbytes = (size_t)window * d.D * esz;
+    const size_t woff = (size_t)(d.L - window) * d.D * esz;
+    if (cudaMemcpy2DAsync(static_cast<char*>(q_dev) + woff, pitch, static_cast<const char*>(q_host) + woff, pitch,
+                          wbytes, (size_t)d.B * d.Hq, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return TSA_ERR_CUDA;
+    float* scores = ws_ptr<float>(ws, w.scores);
+    int32_t* perm = ws_ptr<int32_t>(ws, w.perm);
+    if ((s = run_score(d, q_dev, k_dev, window, scores, ws, st)) != TSA_OK) return s;
+    if ((s = run_select(d, scores, kb, perm, ws, st)) != TSA_OK) return s;
+    if ((s = cuda_status(launch_gather_kept_rows(d, q_map, v_map, perm, kb, q_dev, v_dev, status_word(ws), st))) !=
+        TSA_OK)
+      return s;
+    if ((s = run_attend(d, q_dev, k_dev, v_dev, perm, kb, out_dev, ws, st)) != TSA_OK) return s;
+  }
   if (cudaMemcpyAsync(out_host, out_dev, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TSA_ERR_CUDA;
   return TSA_OK;
+}
+
+size_t tsa_forward_host_h2d_bytes(const tsa_desc* desc, int32_t window, const int32_t* budget_host,
+                                  const void* q_host, const void* v_host) {
+  Dims d;
+  if (check_desc(desc, &d) != TSA_OK || check_window(d, window) != TSA_OK) return 0;
+  Budgets kb;
+  if (load_budgets(d, budget_host, &kb) != TSA_OK) return 0;
+  const void* q_map = q_host ? mapped_device_ptr(q_host) : nullptr;
+  const void* v_map = v_host ? mapped_device_ptr(v_host) : nullptr;
+  const bool sparse = q_map != nullptr && v_map != nullptr && aligned16(q_map) && aligned16(v_map);
+  return host_h2d_bytes(d, window, kb, sparse);
 }
 
 tsa_status tsa_check_status(void* ws, size_t ws_bytes, void* stream) {

@@ -107,6 +107,19 @@ def test_forward_rejects_before_launch(lib):
                                 1 << 40, None) == N.STATUS["TSA_ERR_INVALID_ARG"]
 
 
+def test_host_h2d_bytes_counts(lib):
+    d = desc()
+    b = N._budgets([4096] * 8)
+    # Plain (pageable) host memory is not mapped into any device: the full-copy count.
+    buf = (ctypes.c_uint8 * 64)()
+    a = ctypes.addressof(buf)
+    n = lib.tsa_forward_host_h2d_bytes(ctypes.byref(d), 64, b, a, a)
+    assert n == (d.B * d.Hq + 2 * d.B * d.Hkv) * d.L * d.D * 2
+    assert lib.tsa_forward_host_h2d_bytes(ctypes.byref(desc(D=96)), 64, b, a, a) == 0
+    assert lib.tsa_forward_host_h2d_bytes(ctypes.byref(d), 0, b, a, a) == 0
+    assert lib.tsa_forward_host_h2d_bytes(ctypes.byref(d), 64, N._budgets([0] * 8), a, a) == 0
+
+
 def test_status_strings(lib):
     for code in range(7):
         assert N.tsa_status_string(code)
