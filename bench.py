@@ -541,8 +541,11 @@ def main():
     flops = block_sparse_flops(w, budgets, bm_host) if block_sparse else attend_flops(w, budgets)
     achieved = flops / (t_attend / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic, traffic_src = kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
-                                                                       "long_context_tsa_b200/csrc/tc_ptx.cuh"])
+    # The committed DRAM capture is of the plain forward's attention launch (fixed budgets, no mask, zero
+    # fill, no accumulate); other ops launch it differently, so they carry no traffic figure.
+    traffic, traffic_src = (kernel_traffic("attend", args.workload, ["long_context_tsa_b200/csrc/attend_tc.cu",
+                                                                        "long_context_tsa_b200/csrc/tc_ptx.cuh"])
+                            if args.op in ("forward", "forward-out-proj") else (None, None))
     op_line = None
     if out_proj:
         if T.tsa_check_status(op_ws) != 0:
