@@ -87,8 +87,8 @@ struct Cfg {
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_IDX = OFF_KV + NS * KV_BYTES;  // row tables: Q tiles (2 x 128), K/V tile (128)
   static constexpr int OFF_BAR = OFF_IDX + 3 * 128 * 4;
-  // barriers: q, full[NS], empty[NS], s[2], p[2], o[2], teardown; then tmem slot, abort flag
-  static constexpr int NBAR = 1 + 2 * NS + 6 + 1;
+  // barriers: q (tile 0), full[NS], empty[NS], s[2], p[2], o[2], teardown, q (tile 1); then tmem slot, abort flag
+  static constexpr int NBAR = 1 + 2 * NS + 6 + 1 + 1;  // + the second Q tile
   static constexpr int OFF_ZERO = (OFF_BAR + NBAR * 8 + 16 + 15) / 16 * 16;  // one row of zeros (bulk-copy source)
   static constexpr int SMEM = OFF_ZERO + D * 2 + 1024;  // + alignment slack
   static constexpr int CPR = D / 8;    // 16-byte chunks per row
@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
   auto bar_p = [&](int t) { return bar0 + 8u * (3 + 2 * C::NS + t); };
   auto bar_o = [&](int t) { return bar0 + 8u * (5 + 2 * C::NS + t); };
   const uint32_t bar_td = bar0 + 8u * (7 + 2 * C::NS);
+  const uint32_t bar_q1 = bar0 + 8u * (8 + 2 * C::NS);  // Q tile 1 (bar_q: Q tile 0)
   int* qtab = reinterpret_cast<int*>(gbase + C::OFF_IDX);          // [2][128] global q rows
   int* kvtab = reinterpret_cast<int*>(gbase + C::OFF_IDX + 1024);  // [128] global k/v rows
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + C::NBAR * 8);
@@ -165,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 32 * kProducerWarps);  // every producer lane arrives once its own copies land
+    mbar_init(bar_q1, 32 * kProducerWarps);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar_full(s), 32 * kProducerWarps);
       mbar_init(bar_empty(s), 1);
@@ -200,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     // whole rows.  After issuing a tile every lane arrives on the tile's
     // barrier through cp.async.mbarrier.arrive, which fires once the lane's
     // copies have landed: no lane waits for its own copies, so loads of every
-    // free ring stage are in flight at once.  The Q tiles arrive on bar_q, ring
+    // free ring stage are in flight at once.  Q tile 0 arrives on bar_q, Q tile 1
+    // (issued right after K_0: the first QK waits only for Q tile 0 and K_0) on bar_q1, ring
     // load i (K_0, V_0, K_1, ...) on full[i % NS]; the MMA thread makes the
     // landed rows visible to the tensor core (proxy fence) after its wait.
     const int pw = warp - kProducerWarp0;  // this warp owns rows [32 pw, 32 pw + 32) of every tile
@@ -224,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
     }
     __syncwarp();
     issue_tile(sQ, p.q, qtab);
-    issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);
     cp_async_mbar_arrive(bar_q);
     const int kv_row0 = (b * p.Hkv + g) * L;
     int kt_load = next_active(-1);  // the active tile whose rows y_next holds
@@ -248,6 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
       }
       issue_tile(sKV + s * C::KV_BYTES, (i & 1) ? p.v : p.k, kvtab);
       cp_async_mbar_arrive(bar_full(s));
+      if (i == 0) {  // Q tile 1 after K_0: the first QK needs only Q tile 0 and K_0
+        issue_tile(sQ + C::Q_BYTES, p.q, qtab + 128);
+        cp_async_mbar_arrive(bar_q1);
+      }
     }
     cp_async_wait_all();  // no copy is still writing shared memory when the CTA exits
   } else if (warp >= kZeroWarp0) {
@@ -311,9 +317,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(const TcAttendParams p)
         tc_fence_after();
         qk(0, 0);
         tc_commit(bar_s(0));
-        qk(1, 0);
-        tc_commit(bar_s(1));
-        tc_commit(bar_empty(0));  // K_0 consumed once both QKs complete
+        ok = mbar_wait(bar_q1, 0, p.wait_limit, abort_flag);
+        fence_proxy_async_smem();
+        if (ok) {
+          tc_fence_after();
+          qk(1, 0);
+          tc_commit(bar_s(1));
+          tc_commit(bar_empty(0));  // K_0 consumed once both QKs complete
+        }
       }
       for (int j = 0; ok && j < n_act; ++j) {  // j counts active tiles
         const int iv = 2 * j + 1, ik_next = 2 * j + 2;
